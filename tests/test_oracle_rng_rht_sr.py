@@ -1,0 +1,150 @@
+"""Pins for the oracle's Philox stream, randomized Hadamard transform and
+stochastic rounding (abstract: "randomized Hadamard transforms, and
+stochastic rounding").  References: curand's host-side Philox4x32-10, the
+closed-form Sylvester matrix, binary64 arithmetic and statistics."""
+import numpy as np
+
+import oracle
+
+
+def test_philox_matches_curand(curand_philox):
+    rng = np.random.default_rng(0)
+    n = 10000
+    ctr = rng.integers(0, 2 ** 32, size=(n, 4), dtype=np.uint64)
+    key = rng.integers(0, 2 ** 32, size=(n, 2), dtype=np.uint64)
+    ctr[:8] = 0
+    key[:8] = 0
+    ctr[8] = 0xFFFFFFFF
+    key[8] = 0xFFFFFFFF
+    ref = curand_philox(ctr, key)
+    ours = np.stack([oracle.philox4x32_10(c, k) for c, k in zip(ctr, key)])
+    assert np.array_equal(ref, ours)
+
+
+def test_sr_bits_are_curand_words(curand_philox):
+    """Element n draws 16 bits of Philox(key=seed, ctr=(n>>3 lo, hi, offset, 0))."""
+    seed, offset = 0x1234_5678_9ABC_DEF0, 7
+    ns = [0, 1, 2, 3, 7, 8, 15, 1 << 33, (1 << 40) + 5]
+    ctr = np.array([[(n >> 3) & 0xFFFFFFFF, (n >> 3) >> 32, offset, 0] for n in ns], dtype=np.uint64)
+    key = np.array([[seed & 0xFFFFFFFF, seed >> 32]] * len(ns), dtype=np.uint64)
+    words = curand_philox(ctr, key)
+    for n, w in zip(ns, words):
+        j = n & 7
+        want = (int(w[j >> 1]) >> (16 * (j & 1))) & 0xFFFF
+        assert oracle.sr_bits16(seed, offset, n) == want
+
+
+def test_rht_signs_are_curand_bits(curand_philox):
+    for seed in (0, 1, 0xDEADBEEF, (1 << 40) + 3):
+        w = curand_philox(np.array([[0, 0, 0, 1]], dtype=np.uint64),
+                          np.array([[seed & 0xFFFFFFFF, seed >> 32]], dtype=np.uint64))[0]
+        want = np.array([-1.0 if (int(w[0]) >> i) & 1 else 1.0 for i in range(16)], dtype=np.float32)
+        assert np.array_equal(oracle.rht_signs(seed), want)
+
+
+def sylvester16():
+    i = np.arange(16)
+    par = np.array([[bin(a & b).count("1") & 1 for b in i] for a in i])
+    return np.where(par == 1, -1.0, 1.0)
+
+
+def test_rht_unit_vectors_give_hadamard_rows():
+    """With all signs +1, e_i maps to row i of H16/4 exactly; H H^T = 16 I."""
+    H = sylvester16()
+    assert np.array_equal(H @ H.T, 16 * np.eye(16))
+    ones = np.ones(16, dtype=np.float32)
+    for i in range(16):
+        e = np.zeros(16, dtype=np.float32)
+        e[i] = 1.0
+        assert np.array_equal(oracle.rht16(e, ones), (H[i] / 4).astype(np.float32))
+
+
+def test_rht_matches_dense_f64_within_rounding_bound():
+    rng = np.random.default_rng(5)
+    u = 2.0 ** -24
+    for _ in range(500):
+        x = (rng.standard_normal(16) * np.exp(rng.uniform(-20, 20))).astype(np.float32)
+        s = np.where(rng.random(16) < 0.5, -1.0, 1.0).astype(np.float32)
+        y = oracle.rht16(x, s).astype(np.float64)
+        yd = oracle.rht16_dense_f64(x.astype(np.float64), s.astype(np.float64))
+        yref = (s.astype(np.float64) * x.astype(np.float64)) @ sylvester16() / 4
+        assert np.allclose(yd, yref, rtol=0, atol=1e-300 + 1e-15 * np.abs(x).sum())
+        bound = 4 * u * np.abs(x.astype(np.float64)).sum() / 4 * (1 + 4 * u)
+        assert np.all(np.abs(y - yref) <= bound)
+
+
+def test_rht_preserves_norm():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((200, 64)).astype(np.float32)
+    y = oracle.rht_rows(x, seed=9).astype(np.float64)
+    nx = np.linalg.norm(x.astype(np.float64).reshape(-1, 16), axis=1)
+    ny = np.linalg.norm(y.reshape(-1, 16), axis=1)
+    assert np.all(np.abs(ny - nx) <= 16 * 2.0 ** -24 * nx + 1e-30)
+
+
+def test_rht_cancels_in_the_product():
+    """(X R)(W R)^T = X W^T: the same signed Hadamard on both operands along
+    the contraction dim leaves the product unchanged (up to fp32 rounding)."""
+    rng = np.random.default_rng(8)
+    X = rng.standard_normal((48, 128)).astype(np.float32)
+    W = rng.standard_normal((40, 128)).astype(np.float32)
+    XR = oracle.rht_rows(X, seed=3).astype(np.float64)
+    WR = oracle.rht_rows(W, seed=3).astype(np.float64)
+    ref = X.astype(np.float64) @ W.astype(np.float64).T
+    bound = 16 * 2.0 ** -24 * (np.abs(X).astype(np.float64) @ np.abs(W).astype(np.float64).T) * 4
+    assert np.all(np.abs(XR @ WR.T - ref) <= bound)
+
+
+def test_rht_butterfly_order_independent_check():
+    """An in-place radix-2 butterfly (strides 1, 2, 4, 8; (a, b) -> (a+b,
+    a-b) in float32) written here with numpy scalars agrees bit for bit with
+    the oracle's product of explicit Kronecker factors."""
+    rng = np.random.default_rng(10)
+    for _ in range(300):
+        x = (rng.standard_normal(16) * np.exp(rng.uniform(-30, 30))).astype(np.float32)
+        x[rng.random(16) < 0.1] = np.float32(0.0)
+        s = np.where(rng.random(16) < 0.5, -1.0, 1.0).astype(np.float32)
+        t = [np.float32(np.float32(si * xi) * np.float32(0.25)) for si, xi in zip(s, x)]
+        h = 1
+        while h < 16:
+            for base in range(0, 16, 2 * h):
+                for i in range(base, base + h):
+                    a, b = t[i], t[i + h]
+                    t[i], t[i + h] = np.float32(a + b), np.float32(a - b)
+            h *= 2
+        y = oracle.rht16(x, s)
+        assert np.array_equal(np.array(t, dtype=np.float32).view(np.uint32), y.view(np.uint32))
+
+
+def test_sr_exhaustive_over_r16():
+    """For fixed v the number of r16 in [0, 2^16) that round up is
+    ceil(f * 2^16): exactly the draws with r16 * 2^-16 < f."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    rng = np.random.default_rng(12)
+    for i in range(7):
+        lo, hi = grid[i], grid[i + 1]
+        for frac in (0.0, 1 / 3, 0.5, 0.9, float(rng.random()), 2.0 ** -20):
+            v = np.float32(lo + frac * (hi - lo))
+            f = (float(v) - lo) / (hi - lo)
+            ups = sum(1 for r in range(0, 65536) if (oracle.e2m1_sr(float(v), r) & 7) == i + 1)
+            assert ups == int(np.ceil(f * 65536))
+
+
+def test_sr_unbiased_over_1e6_draws():
+    """Mean of dequantised SR values equals v within 5 sigma plus the 2^-16
+    resolution bias, for v at fractions {1/3, 0.5, 0.9} of each interval."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    rows = 32768                               # 31 draws per row -> ~1.0e6 draws
+    for i in range(7):
+        lo, hi = grid[i], grid[i + 1]
+        for frac in (1 / 3, 0.5, 0.9):
+            v = np.float32(lo + frac * (hi - lo))
+            x = np.full((rows, 32), v, dtype=np.float32)
+            x[:, 0] = 6.0                      # fixes the block scale at 1
+            codes, scales = oracle.quantize_1d(x, sr=True, sr_seed=99, sr_offset=i)
+            assert np.all(scales == 127)
+            deq = oracle.dequant_1d(codes, scales)[:, 1:]
+            n = deq.size
+            p = (float(v) - lo) / (hi - lo)
+            sigma = (hi - lo) * np.sqrt(p * (1 - p) / n)
+            assert abs(deq.mean() - float(v)) <= 5 * sigma + (hi - lo) * 2.0 ** -16
