@@ -1,0 +1,405 @@
+// mxfp4_api.cu -- the C ABI of libmxfp4 (declared in include/mxfp4.h):
+// argument validation, tensor-map encoding and kernel launches on the
+// caller's stream.  No allocation, no exceptions across the boundary.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "../../include/mxfp4.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "quantize.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+__device__ uint32_t g_device_status;
+
+mxfp4_status fail(mxfp4_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+mxfp4_status ok() { return MXFP4_OK; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mxfp4_status check_launch(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+uint32_t* status_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    return static_cast<uint32_t*>(p);
+}
+
+// Host-side Philox4x32-10 (SC'11 constants) for the RHT sign word: bit i of
+// word 0 of Philox(key = seed, counter = (0, 0, 0, 1)).
+uint32_t rht_sign_mask(uint64_t seed) {
+    uint32_t c[4] = {0u, 0u, 0u, 1u};
+    uint32_t k0 = uint32_t(seed), k1 = uint32_t(seed >> 32);
+    for (int round = 0; round < 10; ++round) {
+        const uint64_t p0 = uint64_t(0xD2511F53u) * c[0];
+        const uint64_t p1 = uint64_t(0xCD9E8D57u) * c[2];
+        const uint32_t n0 = uint32_t(p1 >> 32) ^ c[1] ^ k0;
+        const uint32_t n2 = uint32_t(p0 >> 32) ^ c[3] ^ k1;
+        c[0] = n0;
+        c[1] = uint32_t(p1);
+        c[2] = n2;
+        c[3] = uint32_t(p0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return c[0] & 0xFFFFu;
+}
+
+unsigned grid_for(int64_t work, int threads) {
+    const int64_t blocks = (work + threads - 1) / threads;
+    const int64_t cap = int64_t(num_sms()) * 16;
+    return unsigned(blocks < 1 ? 1 : (blocks > cap ? cap : blocks));
+}
+
+// --- quantisation launchers --------------------------------------------------
+template <typename InT>
+mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
+    const int64_t work = qa.groups * qa.rows * (qa.cols / 16);
+    const unsigned grid = grid_for(work, 256);
+    if (rht && sr) mxfp4::quant1d_rows_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);
+    else if (rht) mxfp4::quant1d_rows_kernel<InT, true, false><<<grid, 256, 0, st>>>(qa);
+    else if (sr) mxfp4::quant1d_rows_kernel<InT, false, true><<<grid, 256, 0, st>>>(qa);
+    else mxfp4::quant1d_rows_kernel<InT, false, false><<<grid, 256, 0, st>>>(qa);
+    return check_launch("mxfp4_quantize(1d)");
+}
+
+template <typename InT>
+mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
+    const dim3 grid(unsigned((qa.rows + mxfp4::kTT - 1) / mxfp4::kTT), unsigned((qa.cols + mxfp4::kTF - 1) / mxfp4::kTF),
+                    unsigned(qa.groups));
+    if (rht && sr) mxfp4::quant1d_cols_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);
+    else if (rht) mxfp4::quant1d_cols_kernel<InT, true, false><<<grid, 256, 0, st>>>(qa);
+    else if (sr) mxfp4::quant1d_cols_kernel<InT, false, true><<<grid, 256, 0, st>>>(qa);
+    else mxfp4::quant1d_cols_kernel<InT, false, false><<<grid, 256, 0, st>>>(qa);
+    return check_launch("mxfp4_quantize(1d along rows)");
+}
+
+template <typename InT, bool DEOSC>
+mxfp4_status launch_2d(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
+    const int64_t nblocks = qa.groups * (qa.rows / 32) * (qa.cols / 32);
+    const unsigned grid = unsigned((nblocks + 7) / 8);
+    if constexpr (DEOSC) {
+        mxfp4::quant2d_kernel<InT, false, false, true><<<grid, 256, 0, st>>>(qa);
+    } else {
+        if (rht && sr) mxfp4::quant2d_kernel<InT, true, true, false><<<grid, 256, 0, st>>>(qa);
+        else if (rht) mxfp4::quant2d_kernel<InT, true, false, false><<<grid, 256, 0, st>>>(qa);
+        else if (sr) mxfp4::quant2d_kernel<InT, false, true, false><<<grid, 256, 0, st>>>(qa);
+        else mxfp4::quant2d_kernel<InT, false, false, false><<<grid, 256, 0, st>>>(qa);
+    }
+    return check_launch(DEOSC ? "mxfp4_deosc_update" : "mxfp4_quantize(2d)");
+}
+
+mxfp4_status check_outputs(const mxfp4_quant_outputs* out, bool two_d) {
+    if (!out || !out->codes) return fail(MXFP4_ERR_INVALID_ARG, "outputs: codes pointer is null");
+    if (!aligned16(out->codes)) return fail(MXFP4_ERR_MISALIGNED, "outputs: codes not 16-byte aligned");
+    if (!two_d && (out->codes_t || out->scales_mma_t))
+        return fail(MXFP4_ERR_INVALID_ARG, "outputs: codes_t / scales_mma_t are for 2D blocks only");
+    if (out->scales_mma_t && !out->codes_t)
+        return fail(MXFP4_ERR_INVALID_ARG, "outputs: scales_mma_t needs codes_t");
+    if (out->codes_t && !aligned16(out->codes_t)) return fail(MXFP4_ERR_MISALIGNED, "outputs: codes_t misaligned");
+    return ok();
+}
+
+// --- tensor maps ---------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[3], s[2];
+    cuuint32_t b[3], e[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+    return fn(m, dt, cuuint32_t(rank), const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mxfp4_mma_scale_bytes(int64_t rows, int64_t nscales) {
+    if (rows <= 0 || nscales <= 0) return 0;
+    return size_t(mxfp4::mma_scale_bytes(rows, nscales));
+}
+
+const char* mxfp4_version(void) { return "mxfp4-b200 0.1 (sm_100a)"; }
+
+size_t mxfp4_last_error(char* buf, size_t len) {
+    const size_t n = g_last_error.size();
+    if (buf && len) {
+        const size_t c = n < len - 1 ? n : len - 1;
+        memcpy(buf, g_last_error.data(), c);
+        buf[c] = 0;
+    }
+    return n;
+}
+
+mxfp4_status mxfp4_check_device_status(void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(v), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "check_device_status: %s", cudaGetErrorString(e));
+    if (v == 0) return ok();
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (v & mxfp4::kStatusTimeout)
+        return fail(MXFP4_ERR_DEVICE_TIMEOUT, "device wait timed out (status 0x%08x: roles %s%s%s%s)", v,
+                    (v & mxfp4::kRoleProducer) ? "producer " : "", (v & mxfp4::kRoleMma) ? "mma " : "",
+                    (v & mxfp4::kRoleEpilogue) ? "epilogue " : "", (v & mxfp4::kRoleTeardown) ? "teardown" : "");
+    return fail(MXFP4_ERR_DEVICE_BAD_INPUT, "device rejected group offsets (status 0x%08x)", v);
+}
+
+mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_t rows, int64_t cols, int64_t ld,
+                            const mxfp4_quant_params* p, const mxfp4_quant_outputs* out, void* stream) {
+    if (!in || !p) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: null input or params");
+    if (in_dtype != MXFP4_DTYPE_BF16 && in_dtype != MXFP4_DTYPE_F32)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad in_dtype %d", in_dtype);
+    if (groups < 0 || rows < 0 || cols < 0 || ld < cols)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad geometry groups=%lld rows=%lld cols=%lld ld=%lld",
+                    (long long)groups, (long long)rows, (long long)cols, (long long)ld);
+    if (p->block != MXFP4_BLOCK_1X32 && p->block != MXFP4_BLOCK_32X32)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad block %d", p->block);
+    if (p->rht_d != 0 && p->rht_d != 16) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: rht_d must be 0 or 16");
+    if (p->rounding != MXFP4_ROUND_NEAREST && p->rounding != MXFP4_ROUND_STOCHASTIC)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad rounding %d", p->rounding);
+    const bool two_d = p->block == MXFP4_BLOCK_32X32;
+    mxfp4_status s = check_outputs(out, two_d);
+    if (s != MXFP4_OK) return s;
+    const bool along_rows = !two_d && p->along_rows;
+    if (two_d) {
+        if (rows % 32 || cols % 32)
+            return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize(2d): rows and cols must be multiples of 32");
+    } else if (along_rows) {
+        if (rows % 32) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize(along rows): rows %% 32 != 0");
+    } else if (cols % 32) {
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize: cols %% 32 != 0");
+    }
+    const int esz = in_dtype == MXFP4_DTYPE_BF16 ? 2 : 4;
+    if (!aligned16(in) || (ld * esz) % 16) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_quantize: input rows not 16-byte aligned");
+    if (groups == 0 || rows == 0 || cols == 0) return ok();
+    mxfp4::QuantArgs qa{};
+    qa.in = in;
+    qa.groups = groups;
+    qa.rows = rows;
+    qa.cols = cols;
+    qa.ld = ld;
+    qa.rht_signs = p->rht_d == 16 ? rht_sign_mask(p->rht_seed) : 0u;
+    qa.sr_key0 = uint32_t(p->sr_seed);
+    qa.sr_key1 = uint32_t(p->sr_seed >> 32);
+    qa.sr_offset = p->sr_offset;
+    qa.codes = out->codes;
+    qa.scales = out->scales;
+    qa.scales_mma = out->scales_mma;
+    qa.codes_t = out->codes_t;
+    qa.scales_mma_t = out->scales_mma_t;
+    const bool rht = p->rht_d == 16, sr = p->rounding == MXFP4_ROUND_STOCHASTIC;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (two_d)
+        return in_dtype == MXFP4_DTYPE_BF16 ? launch_2d<uint16_t, false>(qa, rht, sr, st)
+                                            : launch_2d<float, false>(qa, rht, sr, st);
+    if (along_rows)
+        return in_dtype == MXFP4_DTYPE_BF16 ? launch_cols<uint16_t>(qa, rht, sr, st) : launch_cols<float>(qa, rht, sr, st);
+    return in_dtype == MXFP4_DTYPE_BF16 ? launch_rows<uint16_t>(qa, rht, sr, st) : launch_rows<float>(qa, rht, sr, st);
+}
+
+mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int d, uint64_t seed,
+                       void* out, int out_dtype, void* stream) {
+    if (!in || !out) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: null pointer");
+    if (d != 16) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: only d = 16 is supported");
+    if ((in_dtype != MXFP4_DTYPE_BF16 && in_dtype != MXFP4_DTYPE_F32) ||
+        (out_dtype != MXFP4_DTYPE_BF16 && out_dtype != MXFP4_DTYPE_F32))
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: bad dtype");
+    if (rows < 0 || cols < 0 || ld < cols) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: bad geometry");
+    if (cols % 16) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_rht: cols %% 16 != 0");
+    const int esz = in_dtype == MXFP4_DTYPE_BF16 ? 2 : 4;
+    if (!aligned16(in) || !aligned16(out) || (ld * esz) % 16)
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_rht: pointers/rows not 16-byte aligned");
+    if (rows == 0 || cols == 0) return ok();
+    const uint32_t signs = rht_sign_mask(seed);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = grid_for(rows * (cols / 16), 256);
+    if (in_dtype == MXFP4_DTYPE_BF16) {
+        if (out_dtype == MXFP4_DTYPE_BF16)
+            mxfp4::rht_kernel<uint16_t, true><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(in), rows, cols, ld, signs, out);
+        else
+            mxfp4::rht_kernel<uint16_t, false><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(in), rows, cols, ld, signs, out);
+    } else {
+        if (out_dtype == MXFP4_DTYPE_BF16)
+            mxfp4::rht_kernel<float, true><<<grid, 256, 0, st>>>(static_cast<const float*>(in), rows, cols, ld, signs, out);
+        else
+            mxfp4::rht_kernel<float, false><<<grid, 256, 0, st>>>(static_cast<const float*>(in), rows, cols, ld, signs, out);
+    }
+    return check_launch("mxfp4_rht");
+}
+
+mxfp4_status mxfp4_deosc_update(const float* master, int64_t groups, int64_t rows, int64_t cols, uint32_t step,
+                                const mxfp4_deosc_params* dp, uint8_t* state, const mxfp4_quant_outputs* out,
+                                void* stream) {
+    if (!master || !state || !dp) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: null pointer");
+    if (dp->flip_threshold < 1 || dp->flip_threshold > 7)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: flip_threshold must be in 1..7");
+    if (groups < 0 || rows < 0 || cols < 0) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: bad geometry");
+    mxfp4_status s = check_outputs(out, true);
+    if (s != MXFP4_OK) return s;
+    if (rows % 32 || cols % 32) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_deosc_update: rows, cols must be multiples of 32");
+    if (!aligned16(master) || !aligned16(state))
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_deosc_update: master/state not 16-byte aligned");
+    if (groups == 0 || rows == 0 || cols == 0) return ok();
+    mxfp4::QuantArgs qa{};
+    qa.in = master;
+    qa.groups = groups;
+    qa.rows = rows;
+    qa.cols = cols;
+    qa.ld = cols;
+    qa.codes = out->codes;
+    qa.scales = out->scales;
+    qa.scales_mma = out->scales_mma;
+    qa.codes_t = out->codes_t;
+    qa.scales_mma_t = out->scales_mma_t;
+    qa.state = state;
+    qa.step = step;
+    qa.flip_threshold = dp->flip_threshold;
+    qa.reset_period = dp->reset_period;
+    return launch_2d<float, true>(qa, false, false, static_cast<cudaStream_t>(stream));
+}
+
+mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_offsets, mxfp4_operand A,
+                                mxfp4_operand B, int64_t M, int64_t N, int64_t K, float* out, int64_t ldo,
+                                void* stream) {
+    using namespace mxfp4::gemm;
+    if (op != MXFP4_GEMM_FPROP && op != MXFP4_GEMM_DGRAD && op != MXFP4_GEMM_WGRAD)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad op %d", op);
+    if (num_groups <= 0 || !group_offsets || !A.codes || !A.scales_mma || !B.codes || !B.scales_mma || !out)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: null pointer or num_groups <= 0");
+    if (M < 0 || N <= 0 || K < 0 || ldo < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad geometry");
+    if (K % 128 && op == MXFP4_GEMM_WGRAD)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm(wgrad): total tokens must be a multiple of 128");
+    if (K % 64) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: K %% 64 != 0");
+    if (op != MXFP4_GEMM_WGRAD && M % 128)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: M must be a multiple of 128 (padded groups)");
+    if (ldo % 4) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: ldo must be a multiple of 4");
+    if (!aligned16(A.codes) || !aligned16(B.codes) || !aligned16(A.scales_mma) || !aligned16(B.scales_mma) ||
+        !aligned16(out) || (reinterpret_cast<uintptr_t>(group_offsets) & 3u))
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: pointer not 16-byte aligned");
+    if (M == 0) return ok();
+    if (K == 0) {
+        if (op != MXFP4_GEMM_WGRAD) return ok();
+        // every group is empty: dW_g = 0
+        const cudaError_t e = cudaMemset2DAsync(out, size_t(ldo) * 4, 0, size_t(N) * 4, size_t(M) * num_groups,
+                                                static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot resolve the device status word");
+
+    Args a{};
+    a.mode = op == MXFP4_GEMM_WGRAD ? 1 : 0;
+    a.num_groups = num_groups;
+    a.offsets = group_offsets;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.sfa = A.scales_mma;
+    a.sfb = B.scales_mma;
+    const int64_t S = (K + 31) / 32;
+    a.nchunk_a = (S + 3) / 4;
+    a.nchunk_b = (S + 3) / 4;
+    a.nrb_b = (N + 127) / 128;
+    a.sfb_group_bytes = mxfp4::mma_scale_bytes(N, S);
+    a.m_tiles = int((M + BM - 1) / BM);
+    a.n_tiles = int((N + BN - 1) / BN);
+    a.total_tiles = a.mode == 0 ? int64_t(a.m_tiles) * a.n_tiles : int64_t(num_groups) * a.m_tiles * a.n_tiles;
+    a.status = status;
+
+    CUtensorMap tmA, tmB, tmD;
+    const uint64_t kb = uint64_t(K / 2);
+    {
+        const uint64_t dims[2] = {kb, uint64_t(M)};
+        const uint64_t str[1] = {kb};
+        const uint32_t box[2] = {128, BM};
+        if (!make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, A.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for A failed");
+    }
+    if (a.mode == 0) {
+        const uint64_t dims[3] = {kb, uint64_t(N), uint64_t(num_groups)};
+        const uint64_t str[2] = {kb, kb * uint64_t(N)};
+        const uint32_t box[3] = {128, BN, 1};
+        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, B.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
+        const uint64_t ddims[2] = {uint64_t(N), uint64_t(M)};
+        const uint64_t dstr[1] = {uint64_t(ldo) * 4};
+        const uint32_t dbox[2] = {32, 32};
+        if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, ddims, dstr, dbox))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
+    } else {
+        const uint64_t dims[2] = {kb, uint64_t(N)};
+        const uint64_t str[1] = {kb};
+        const uint32_t box[2] = {128, BN};
+        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, B.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
+        const uint64_t ddims[3] = {uint64_t(N), uint64_t(M), uint64_t(num_groups)};
+        const uint64_t dstr[2] = {uint64_t(ldo) * 4, uint64_t(ldo) * 4 * uint64_t(M)};
+        const uint32_t dbox[3] = {32, 32, 1};
+        if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, ddims, dstr, dbox))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
+    }
+    if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+        return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
+    if (a.total_tiles == 0) return ok();
+    const int64_t sms = num_sms();
+    const unsigned grid = unsigned(a.total_tiles < sms ? a.total_tiles : sms);
+    grouped_gemm_kernel<<<grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, a);
+    return check_launch("mxfp4_grouped_gemm");
+}
+
+}  // extern "C"

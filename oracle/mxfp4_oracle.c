@@ -181,7 +181,7 @@ int oracle_e2m1_sr(float v, uint32_t r16)
 
 /* ------------------------------------------------------------------------ */
 /* Randomized Hadamard transform on one 16-element chunk (reading of the    */
-/* "randomized Hadamard transforms" of the abstract, d = 16):               */
+/* RHT the abstract names, with d = 16):                                     */
 /*   t = (s .* x) * 1/4            (exact)                                   */
 /*   y = t * F1 * F2 * F4 * F8     each factor applied in binary32           */
 /* where F_h = I_{16/2h} (x) H2 (x) I_h with H2 = [[1,1],[1,-1]].  Each      */
@@ -405,8 +405,8 @@ void oracle_quantize_2d(const void* in, int dtype, int64_t rows, int64_t cols, i
 
 /* ------------------------------------------------------------------------ */
 /* Weight de-oscillation (reading; the pages give the motivation on         */
-/* roboaidigest "What ALTO Actually Does" and the name "simplified,         */
-/* adapted from TetraJet-v2" in the abstract, not the rule).                 */
+/* roboaidigest "What ALTO Actually Does"; the abstract says only that the  */
+/* scheme is a simplified one derived from TetraJet-v2, not the rule).       */
 /* Per weight, one state byte: bits 0-3 previous code, bits 4-6 flip count  */
 /* (saturating at 7), bit 7 frozen.                                          */
 /*  step == 0 : initialise state = (RN code, count 0, not frozen).           */

@@ -1,0 +1,80 @@
+"""CPU checks of the boundary: libmxfp4.so builds for sm_100a, loads, and
+exports every entry point include/mxfp4.h declares; host-side argument
+validation runs without a GPU (no compute call is made)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mxfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def libpath():
+    from fp4_precision_numerics_b200 import build
+    return build.build()
+
+
+def test_header_declares_the_four_calls():
+    fns = declared_functions()
+    for name in ("mxfp4_quantize", "mxfp4_rht", "mxfp4_deosc_update", "mxfp4_grouped_gemm"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(libpath):
+    out = subprocess.run(["nm", "-D", "--defined-only", libpath], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)", out))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    # nothing else leaks out with the mxfp4_ prefix
+    extra = [s for s in exported if s.startswith("mxfp4_") and s not in declared_functions()]
+    assert not extra, extra
+
+
+def test_library_loads_and_reports_version(libpath):
+    L = ctypes.CDLL(libpath)
+    L.mxfp4_version.restype = ctypes.c_char_p
+    assert b"sm_100a" in L.mxfp4_version()
+    L.mxfp4_mma_scale_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    L.mxfp4_mma_scale_bytes.restype = ctypes.c_size_t
+    assert L.mxfp4_mma_scale_bytes(128, 4) == 512
+    assert L.mxfp4_mma_scale_bytes(2880, 90) == 23 * 23 * 512
+    assert L.mxfp4_mma_scale_bytes(0, 4) == 0
+
+
+def test_host_validation_without_gpu(libpath):
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    p = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 0, 0, 0, 0, 0, 0)
+    o = mxfp4.QuantOutputs(None, None, None, None, None)
+    # null input
+    assert L.mxfp4_quantize(None, 0, 1, 4, 32, 32, ctypes.byref(p), ctypes.byref(o), None) == -1
+    # null codes output
+    assert L.mxfp4_quantize(ctypes.c_void_p(16), 0, 1, 4, 32, 32, ctypes.byref(p), ctypes.byref(o), None) == -1
+    o.codes = 16
+    # cols not a multiple of 32
+    assert L.mxfp4_quantize(ctypes.c_void_p(16), 0, 1, 4, 48, 48, ctypes.byref(p), ctypes.byref(o), None) == -2
+    # misaligned input
+    assert L.mxfp4_quantize(ctypes.c_void_p(18), 0, 1, 4, 32, 32, ctypes.byref(p), ctypes.byref(o), None) == -3
+    # bad enum
+    p.rounding = 9
+    assert L.mxfp4_quantize(ctypes.c_void_p(16), 0, 1, 4, 32, 32, ctypes.byref(p), ctypes.byref(o), None) == -1
+    assert "rounding" in mxfp4.last_error()
+    # rht with unsupported d
+    assert L.mxfp4_rht(ctypes.c_void_p(16), 0, 4, 32, 32, 8, 0, ctypes.c_void_p(16), 1, None) == -1
+    # gemm: bad op, null operands
+    a = mxfp4.Operand(None, None)
+    assert L.mxfp4_grouped_gemm(7, 1, ctypes.c_void_p(16), a, a, 128, 192, 128, ctypes.c_void_p(16), 192, None) == -1
+    assert L.mxfp4_grouped_gemm(0, 1, ctypes.c_void_p(16), a, a, 128, 192, 128, ctypes.c_void_p(16), 192, None) == -1
+    d = mxfp4.DeoscParams(9, 0)
+    assert L.mxfp4_deosc_update(ctypes.c_void_p(16), 1, 32, 32, 0, ctypes.byref(d), ctypes.c_void_p(16),
+                                ctypes.byref(o), None) == -1

@@ -1,7 +1,7 @@
 """Pins for the oracle's Philox stream, randomized Hadamard transform and
-stochastic rounding (abstract: "randomized Hadamard transforms, and
-stochastic rounding").  References: curand's host-side Philox4x32-10, the
-closed-form Sylvester matrix, binary64 arithmetic and statistics."""
+stochastic rounding (both named by the abstract as recipe techniques).
+References: curand's host-side Philox4x32-10, the closed-form Sylvester
+matrix, binary64 arithmetic and statistics."""
 import numpy as np
 
 import oracle
