@@ -1,0 +1,549 @@
+"""Benchmark: one MXFP4 training step of a GPT-OSS-20B-shaped MoE expert
+layer through libmxfp4 (the ALTO recipe's quantise-and-contract hot path).
+
+A step, all on one GPU and one stream:
+  1. de-oscillation re-quantisation of the fp32 master weights W_up
+     [32, 5760, 2880] and W_down [32, 2880, 2880] (2D 32x32 blocks; emits W
+     and W^T codes and tensor-core scales),
+  2. quantise X and H (1x32 along K, nearest) -> fprop GEMMs Y_up, Y_down,
+  3. quantise dY_up, dY_down (1x32 along N, SR) -> dgrad GEMMs dX, dH,
+  4. quantise X^T, H^T, dY_up^T, dY_down^T along tokens (RHT-16; SR on
+     gradients) -> wgrad GEMMs dW_up, dW_down (fp32).
+16384 tokens routed top-4 over 32 experts with Zipf(1.1) skew (65536 routed
+rows, segments padded to 128).  Inputs are synthetic (seeded), bigger than
+L2, resident in HBM when the timed region starts.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torchrun (one process per GPU); every rank runs its
+own replica of the layer (the path has no exchange step), so per-GPU work is
+fixed and the result line reports weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MXFP4 grouped-GEMM TFLOPS + quantise GB/s, % of FP4/HBM roofline, 1 B200"
+WORKLOAD = ("GPT-OSS-20B-shaped MoE expert layer, full MXFP4 training step (fprop + dgrad + wgrad, "
+            "2D de-oscillation weight re-quantisation), 32 experts, d_model 2880, W_up 5760x2880, "
+            "W_down 2880x2880, 16384 tokens top-4 Zipf(1.1)")
+E, D, F = 32, 2880, 5760
+NOMINAL_FP4_OVER_BF16 = 4.0          # dense FP4 / dense BF16 tensor rate, B200 datasheet (9 / 2.25 PFLOP/s)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=float(j["hbm_gbs"]), bf16_burst=float(j["bf16_tflops"]),
+                    bf16_sustained=float(j.get("bf16_tflops_sustained", j["bf16_tflops"])), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_burst=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# Workload
+# ---------------------------------------------------------------------------
+class Layer:
+    """Device buffers of one MoE layer replica and its training step."""
+
+    def __init__(self, dev, seed=0, n_experts=32, n_tokens=16384):
+        import numpy as np
+        import torch
+
+        from fp4_precision_numerics_b200 import mxfp4, synth
+        self.mx = mxfp4
+        global E
+        E = n_experts
+        self.n_tokens = n_tokens
+        routing = synth.zipf_routing(n_tokens=n_tokens, n_experts=n_experts, seed=2)
+        counts, offsets, tor = synth.expert_layout(routing, n_experts)
+        self.counts = counts
+        self.M = int(offsets[-1])
+        self.rows_real = int(counts.sum())
+        self.offsets = torch.tensor(offsets.astype(np.int32), device=dev)
+        M = self.M
+        g = torch.Generator(device=dev)
+        g.manual_seed(1000 + seed)
+        pad = torch.from_numpy(tor < 0).to(dev)
+
+        def act(shape, std):
+            t = torch.randn(shape, generator=g, device=dev, dtype=torch.float32).mul_(std).to(torch.bfloat16)
+            t[pad] = 0
+            return t
+
+        # token activations are gathered into expert order (each token appears top-4 times)
+        x_tok = torch.randn((n_tokens, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        idx = torch.from_numpy(np.where(tor < 0, 0, tor)).to(dev)
+        self.x = x_tok[idx]
+        self.x[pad] = 0
+        self.h = act((M, D), 1.0)
+        self.dy_up = act((M, F), 1e-3)
+        self.dy_down = act((M, D), 1e-3)
+        self.w_up = torch.randn((E, F, D), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+        self.w_down = torch.randn((E, D, D), generator=g, device=dev, dtype=torch.float32).mul_(0.02)
+        self.st_up = torch.zeros((E, F, D), dtype=torch.uint8, device=dev)
+        self.st_down = torch.zeros((E, D, D), dtype=torch.uint8, device=dev)
+        u8 = dict(dtype=torch.uint8, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        sb = mxfp4.mxfp4_mma_scale_bytes
+        self.q = {
+            "w_up": dict(codes=torch.empty((E, F, D // 2), **u8), scales_mma=torch.empty((E, sb(F, D // 32)), **u8),
+                         codes_t=torch.empty((E, D, F // 2), **u8), scales_mma_t=torch.empty((E, sb(D, F // 32)), **u8)),
+            "w_down": dict(codes=torch.empty((E, D, D // 2), **u8), scales_mma=torch.empty((E, sb(D, D // 32)), **u8),
+                           codes_t=torch.empty((E, D, D // 2), **u8), scales_mma_t=torch.empty((E, sb(D, D // 32)), **u8)),
+            "x": dict(codes=torch.empty((1, M, D // 2), **u8), scales_mma=torch.empty((1, sb(M, D // 32)), **u8)),
+            "h": dict(codes=torch.empty((1, M, D // 2), **u8), scales_mma=torch.empty((1, sb(M, D // 32)), **u8)),
+            "dy_up": dict(codes=torch.empty((1, M, F // 2), **u8), scales_mma=torch.empty((1, sb(M, F // 32)), **u8)),
+            "dy_down": dict(codes=torch.empty((1, M, D // 2), **u8), scales_mma=torch.empty((1, sb(M, D // 32)), **u8)),
+            "xt": dict(codes=torch.empty((1, D, M // 2), **u8), scales_mma=torch.empty((1, sb(D, M // 32)), **u8)),
+            "ht": dict(codes=torch.empty((1, D, M // 2), **u8), scales_mma=torch.empty((1, sb(D, M // 32)), **u8)),
+            "dy_up_t": dict(codes=torch.empty((1, F, M // 2), **u8), scales_mma=torch.empty((1, sb(F, M // 32)), **u8)),
+            "dy_down_t": dict(codes=torch.empty((1, D, M // 2), **u8), scales_mma=torch.empty((1, sb(D, M // 32)), **u8)),
+        }
+        self.y_up = torch.empty((M, F), **f32)
+        self.y_down = torch.empty((M, D), **f32)
+        self.dx = torch.empty((M, D), **f32)
+        self.dh = torch.empty((M, D), **f32)
+        self.dw_up = torch.empty((E, F, D), **f32)
+        self.dw_down = torch.empty((E, D, D), **f32)
+        self.step_idx = 0
+        self.launches_per_step = 16
+        # algorithmic work
+        r = self.rows_real
+        self.gemm_flops = {
+            "fprop_up": 2.0 * r * F * D, "fprop_down": 2.0 * r * D * D,
+            "dgrad_up": 2.0 * r * F * D, "dgrad_down": 2.0 * r * D * D,
+            "wgrad_up": 2.0 * r * F * D, "wgrad_down": 2.0 * r * D * D,
+        }
+        # quantise bytes: read input, write codes (1/2 B) + scales (1/32 B); de-osc adds state r/w
+        q1 = 2.0 + 0.5 + 1.0 / 32
+        self.quant_bytes = {
+            "deosc_up": E * F * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
+            "deosc_down": E * D * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
+            "quant_x": M * D * q1, "quant_h": M * D * q1, "quant_dy_up": M * F * q1, "quant_dy_down": M * D * q1,
+            "quant_xt": M * D * q1, "quant_ht": M * D * q1, "quant_dy_up_t": M * F * q1, "quant_dy_down_t": M * D * q1,
+        }
+        self.gemm_dims = {
+            "fprop_up": (M, F, D), "fprop_down": (M, D, D), "dgrad_up": (M, D, F), "dgrad_down": (M, D, D),
+            "wgrad_up": (F, D, M), "wgrad_down": (D, D, M),
+        }
+
+    def gemm_out_bytes(self, name):
+        """Algorithmic HBM bytes of one GEMM launch: each operand's codes and
+        scales read once, the binary32 output written once."""
+        Mg, N, K = self.gemm_dims[name]
+        per = 0.5 + 1.0 / 32
+        if name.startswith("wgrad"):
+            return (Mg + N) * K * per + E * Mg * N * 4
+        return (Mg * K + E * N * K) * per + Mg * N * 4
+
+    def step(self, ev=None):
+        """One training step.  `ev` (optional) maps a kernel name to a pair of
+        CUDA events recorded around its launch on the current stream."""
+        mx = self.mx
+        q = self.q
+
+        def rec(name, i):
+            if ev is not None:
+                ev[name][i].record()
+
+        s = self.step_idx
+        rec("deosc_up", 0)
+        mx.deosc_update(self.w_up, s, self.st_up, scales=False, scales_mma=True, transposed=True, out=q["w_up"])
+        rec("deosc_up", 1)
+        rec("deosc_down", 0)
+        mx.deosc_update(self.w_down, s, self.st_down, scales=False, scales_mma=True, transposed=True,
+                        out=q["w_down"])
+        rec("deosc_down", 1)
+        M = self.M
+        rec("quant_x", 0)
+        mx.quantize(self.x, scales=False, scales_mma=True, out=q["x"])
+        rec("quant_x", 1)
+        rec("fprop_up", 0)
+        mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["x"]["codes"], q["x"]["scales_mma"], q["w_up"]["codes"],
+                        q["w_up"]["scales_mma"], M, F, D, out=self.y_up)
+        rec("fprop_up", 1)
+        rec("quant_h", 0)
+        mx.quantize(self.h, scales=False, scales_mma=True, out=q["h"])
+        rec("quant_h", 1)
+        rec("fprop_down", 0)
+        mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["h"]["codes"], q["h"]["scales_mma"], q["w_down"]["codes"],
+                        q["w_down"]["scales_mma"], M, D, D, out=self.y_down)
+        rec("fprop_down", 1)
+        rec("quant_dy_up", 0)
+        mx.quantize(self.dy_up, sr_seed=1, sr_offset=2 * s, scales=False, scales_mma=True, out=q["dy_up"])
+        rec("quant_dy_up", 1)
+        rec("dgrad_up", 0)
+        mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_up"]["codes"], q["dy_up"]["scales_mma"],
+                        q["w_up"]["codes_t"], q["w_up"]["scales_mma_t"], M, D, F, out=self.dx)
+        rec("dgrad_up", 1)
+        rec("quant_dy_down", 0)
+        mx.quantize(self.dy_down, sr_seed=1, sr_offset=2 * s + 1, scales=False, scales_mma=True, out=q["dy_down"])
+        rec("quant_dy_down", 1)
+        rec("dgrad_down", 0)
+        mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_down"]["codes"], q["dy_down"]["scales_mma"],
+                        q["w_down"]["codes_t"], q["w_down"]["scales_mma_t"], M, D, D, out=self.dh)
+        rec("dgrad_down", 1)
+        rec("quant_xt", 0)
+        mx.quantize(self.x, along_rows=True, rht_seed=1, scales=False, scales_mma=True, out=q["xt"])
+        rec("quant_xt", 1)
+        rec("quant_dy_up_t", 0)
+        mx.quantize(self.dy_up, along_rows=True, rht_seed=1, sr_seed=1, sr_offset=1000 + 2 * s, scales=False,
+                    scales_mma=True, out=q["dy_up_t"])
+        rec("quant_dy_up_t", 1)
+        rec("wgrad_up", 0)
+        mx.grouped_gemm(mx.GEMM_WGRAD, self.offsets, q["dy_up_t"]["codes"], q["dy_up_t"]["scales_mma"],
+                        q["xt"]["codes"], q["xt"]["scales_mma"], F, D, M, out=self.dw_up)
+        rec("wgrad_up", 1)
+        rec("quant_ht", 0)
+        mx.quantize(self.h, along_rows=True, rht_seed=1, scales=False, scales_mma=True, out=q["ht"])
+        rec("quant_ht", 1)
+        rec("quant_dy_down_t", 0)
+        mx.quantize(self.dy_down, along_rows=True, rht_seed=1, sr_seed=1, sr_offset=1001 + 2 * s, scales=False,
+                    scales_mma=True, out=q["dy_down_t"])
+        rec("quant_dy_down_t", 1)
+        rec("wgrad_down", 0)
+        mx.grouped_gemm(mx.GEMM_WGRAD, self.offsets, q["dy_down_t"]["codes"], q["dy_down_t"]["scales_mma"],
+                        q["ht"]["codes"], q["ht"]["scales_mma"], D, D, M, out=self.dw_down)
+        rec("wgrad_down", 1)
+        self.step_idx += 1
+
+
+KERNELS = ["deosc_up", "deosc_down", "quant_x", "fprop_up", "quant_h", "fprop_down", "quant_dy_up", "dgrad_up",
+           "quant_dy_down", "dgrad_down", "quant_xt", "quant_dy_up_t", "wgrad_up", "quant_ht", "quant_dy_down_t",
+           "wgrad_down"]
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0, t1):
+        rows = [s for (t, s) in self.samples if t0 - 0.05 <= t <= t1 + 0.05] or [s for (_, s) in self.samples]
+        mhz, maxmhz, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                mhz.append(float(parts[0]))
+                maxmhz.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus and world > 1:
+        raise SystemExit("WORLD_SIZE %d != --gpus %d" % (world, n_gpus))
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local, pg
+
+
+def max_over_ranks(value, pg, device):
+    """Max of a float over all ranks (identity for one rank)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle on a bounded sample of the same step
+# ---------------------------------------------------------------------------
+def cpu_baseline_sample(rows=256, expert=0):
+    """Time the oracle (as it stands) on a bounded sample of the step: the
+    first `rows` routed rows of one expert through the up-projection's three
+    GEMMs with the quantisations they need (1x32 X, SR dY, 2D W with
+    de-oscillation state, RHT-16 transposed operands for wgrad).  Returns
+    (TFLOP/s of GEMM work over the sample's wall time, seconds, threads)."""
+    import numpy as np
+
+    import oracle
+    from fp4_precision_numerics_b200 import synth
+    rng = np.random.default_rng(0)
+    x = synth.bf16_bits(rng.standard_normal((rows, D)).astype(np.float32))
+    dy = synth.bf16_bits((rng.standard_normal((rows, F)) * 1e-3).astype(np.float32))
+    w = (rng.standard_normal((F, D)) * 0.02).astype(np.float32)
+    oracle.lib()
+    t0 = time.perf_counter()
+    st = np.zeros((1, F, D), dtype=np.uint8)
+    cw, sw = oracle.deosc_update(w[None], 0, st)
+    Wq = oracle.dequant_2d(cw[0], sw[0])
+    cx, sx = oracle.quantize_1d(x)
+    Xq = oracle.dequant_1d(cx, sx)
+    y = oracle.gemm_f64(Xq, Wq)                                        # fprop
+    cdy, sdy = oracle.quantize_1d(dy, sr=True, sr_seed=1)
+    dYq = oracle.dequant_1d(cdy, sdy)
+    dx = dYq @ Wq                                                      # dgrad (binary64)
+    cxt, sxt = oracle.quantize_1d_transposed(x, rht_d=16, rht_seed=1)
+    cdt, sdt = oracle.quantize_1d_transposed(dy, rht_d=16, rht_seed=1, sr=True, sr_seed=1)
+    dw = oracle.gemm_f64(oracle.dequant_1d(cdt, sdt), oracle.dequant_1d(cxt, sxt))   # wgrad
+    secs = time.perf_counter() - t0
+    del y, dx, dw
+    flops = 3 * 2.0 * rows * F * D
+    return flops / secs / 1e12, secs, oracle.num_threads(), flops
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    samples = []
+    threads = None
+    flops = None
+    for _ in range(args.warmup):
+        cpu_baseline_sample(rows=64)
+    t_all = 0.0
+    for _ in range(args.steps):
+        v, secs, threads, flops = cpu_baseline_sample(rows=64)
+        samples.append(v)
+        t_all += secs
+    value = sum(flops for _ in samples) / t_all / 1e12
+    sample = ("oracle on 64 routed rows of expert 0 per step: up-projection fprop/dgrad/wgrad binary64 GEMMs "
+              "plus the quantisations they need (5760x2880 W with de-oscillation)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t_all / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD + " (bounded CPU sample)", "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Main (our arm)
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=32,
+                    help="smaller layers are for profiler captures only; the result line names the size")
+    ap.add_argument("--tokens", type=int, default=16384)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    rank, world, local, pg = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    peaks = load_peaks()
+    layer = Layer(dev, seed=rank, n_experts=args.experts, n_tokens=args.tokens)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        layer.step()
+    layer.mx.mxfp4_check_device_status()
+    torch.cuda.synchronize()
+
+    # per-kernel events over the timed steps
+    evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
+           for _ in range(args.steps)]
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        gpu_uuid = str(local)
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(pg)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        layer.step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(pg)
+    clocks.stop()
+    layer.mx.mxfp4_check_device_status()
+    ms_local = start.elapsed_time(end)
+    ms = max_over_ranks(ms_local, pg, dev)
+
+    per_kernel = {k: statistics.mean(e[k][0].elapsed_time(e[k][1]) for e in evs) for k in KERNELS}
+    step_flops = sum(layer.gemm_flops.values())
+    value = step_flops * args.steps * world / (ms / 1e3) / 1e12
+    gemm_ms = sum(per_kernel[k] for k in layer.gemm_flops)
+    quant_ms = sum(per_kernel[k] for k in layer.quant_bytes)
+    quant_gbs = sum(layer.quant_bytes.values()) / (quant_ms / 1e3) / 1e9
+    fp4_peak = peaks["bf16_sustained"] * NOMINAL_FP4_OVER_BF16
+    dominant = max(per_kernel, key=lambda k: per_kernel[k])
+    dom_ms = per_kernel[dominant]
+    if dominant in layer.gemm_flops:
+        achieved = layer.gemm_flops[dominant] / (dom_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak,
+                "peak_source": "%s sustained bf16 x %.0f (nominal FP4:BF16 dense ratio)" % (peaks["source"],
+                                                                                          NOMINAL_FP4_OVER_BF16),
+                "kernel": dominant, "traffic": None,
+                "hbm_frac": layer.gemm_out_bytes(dominant) / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    else:
+        achieved = layer.quant_bytes[dominant] / (dom_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
+                "kernel": dominant, "traffic": None}
+    components = {}
+    for k in KERNELS:
+        t = per_kernel[k]
+        if k in layer.gemm_flops:
+            tf = layer.gemm_flops[k] / (t / 1e3) / 1e12
+            gbs = layer.gemm_out_bytes(k) / (t / 1e3) / 1e9
+            components[k] = {"ms": round(t, 4), "tflops": round(tf, 1), "frac_fp4": round(tf / fp4_peak, 4),
+                             "alg_gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+        else:
+            gbs = layer.quant_bytes[k] / (t / 1e3) / 1e9
+            components[k] = {"ms": round(t, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+
+    # ---------------- end to end through the C ABI with host buffers
+    h2d_bytes = sum(t.numel() * t.element_size() for t in (layer.x, layer.h, layer.dy_up, layer.dy_down))
+    host_in = [t.cpu().pin_memory() for t in (layer.x, layer.h, layer.dy_up, layer.dy_down)]
+    host_out = [torch.empty(layer.dx.shape, dtype=torch.float32).pin_memory(),
+                torch.empty(layer.dh.shape, dtype=torch.float32).pin_memory()]
+    d2h_bytes = sum(t.numel() * t.element_size() for t in host_out)
+    dev_in = (layer.x, layer.h, layer.dy_up, layer.dy_down)
+    layer.step()
+    torch.cuda.synchronize()
+    barrier(pg)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        layer.step()
+        host_out[0].copy_(layer.dx, non_blocking=True)
+        host_out[1].copy_(layer.dh, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(pg)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+    e2e_value = step_flops * args.e2e_steps * world / (e2e_ms / 1e3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, secs, threads, _ = cpu_baseline_sample(rows=256)
+        cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": "256 routed rows of expert 0: up-projection fprop/dgrad/wgrad binary64 GEMMs plus their "
+                         "quantisations (2D de-oscillation W, SR dY, RHT-16 transposed operands); %.1f s on %d "
+                         "threads of %d host cores" % (secs, threads, os.cpu_count() or 0)}
+    ck = clocks.summary(t0, t1)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e2m1+ue8m0 (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": WORKLOAD if (args.experts, args.tokens) == (32, 16384) else
+                   "reduced MoE layer for profiling: %d experts, %d tokens" % (args.experts, args.tokens),
+                   "tokens": args.tokens, "routed_rows": layer.rows_real, "padded_rows": layer.M,
+                   "experts": E, "parallelism": "replica per GPU" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (working set ~14 GB per step)"},
+        "quantise_gbs": quant_gbs, "quantise_frac_hbm": quant_gbs / peaks["hbm_gbs"],
+        "gemm_tflops": step_flops / (gemm_ms / 1e3) / 1e12, "gemm_frac_fp4": step_flops / (gemm_ms / 1e3) / 1e12 / fp4_peak,
+        "roofline": roof, "components": components,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d_bytes),
+                "d2h_bytes_per_step": int(d2h_bytes)},
+        "gpu_launches": layer.launches_per_step * args.steps,
+        "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"], "reasons": ck["reasons"],
+                   "samples": ck["samples"]},
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

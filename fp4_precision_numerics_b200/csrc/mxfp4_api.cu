@@ -199,18 +199,21 @@ mxfp4_status mxfp4_check_device_status(void* stream) {
 
 mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_t rows, int64_t cols, int64_t ld,
                             const mxfp4_quant_params* p, const mxfp4_quant_outputs* out, void* stream) {
-    if (!in || !p) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: null input or params");
+    if (!p) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: null params");
     if (in_dtype != MXFP4_DTYPE_BF16 && in_dtype != MXFP4_DTYPE_F32)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad in_dtype %d", in_dtype);
     if (groups < 0 || rows < 0 || cols < 0 || ld < cols)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad geometry groups=%lld rows=%lld cols=%lld ld=%lld",
                     (long long)groups, (long long)rows, (long long)cols, (long long)ld);
+    const bool empty = groups == 0 || rows == 0 || cols == 0;
+    if (!in && !empty) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: null input");
     if (p->block != MXFP4_BLOCK_1X32 && p->block != MXFP4_BLOCK_32X32)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad block %d", p->block);
     if (p->rht_d != 0 && p->rht_d != 16) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: rht_d must be 0 or 16");
     if (p->rounding != MXFP4_ROUND_NEAREST && p->rounding != MXFP4_ROUND_STOCHASTIC)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize: bad rounding %d", p->rounding);
     const bool two_d = p->block == MXFP4_BLOCK_32X32;
+    if (empty) return ok();  // nothing to read or write; output pointers may be null
     mxfp4_status s = check_outputs(out, two_d);
     if (s != MXFP4_OK) return s;
     const bool along_rows = !two_d && p->along_rows;
@@ -224,7 +227,6 @@ mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_
     }
     const int esz = in_dtype == MXFP4_DTYPE_BF16 ? 2 : 4;
     if (!aligned16(in) || (ld * esz) % 16) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_quantize: input rows not 16-byte aligned");
-    if (groups == 0 || rows == 0 || cols == 0) return ok();
     mxfp4::QuantArgs qa{};
     qa.in = in;
     qa.groups = groups;

@@ -166,7 +166,8 @@ def quantize(x: torch.Tensor, block: str = "1x32", along_rows: bool = False, rht
     and tensor-core scales).  `out` may supply preallocated tensors."""
     if x.dim() == 2:
         x = x.unsqueeze(0)
-    assert x.is_cuda and x.dim() == 3 and x.stride(2) == 1 and x.stride(0) == x.shape[1] * x.stride(1)
+    assert x.is_cuda and x.dim() == 3 and x.stride(2) == 1
+    assert x.shape[0] == 1 or x.stride(0) == x.shape[1] * x.stride(1), "groups must be back to back"
     G, R, C = x.shape
     ld = x.stride(1)
     two_d = block == "32x32"
@@ -208,7 +209,9 @@ def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_thre
                  out: dict | None = None, stream=None) -> dict:
     if master.dim() == 2:
         master = master.unsqueeze(0)
-    assert master.dtype == torch.float32 and master.is_contiguous()
+    assert master.dtype == torch.float32 and master.stride(-1) == 1
+    assert master.shape[0] == 1 or master.stride(0) == master.shape[1] * master.shape[2]
+    assert master.stride(1) == master.shape[2]
     assert state.dtype == torch.uint8 and state.is_contiguous() and state.numel() == master.numel()
     G, R, C = master.shape
     o = dict(out or {})

@@ -136,7 +136,7 @@ def test_grouped_rows_share_one_sr_stream():
 
 
 # ----------------------------------------------------------- along the token dim
-@pytest.mark.parametrize("shape", [(256, 192), (1024, 2880), (384, 100), (96, 64)])
+@pytest.mark.parametrize("shape", [(256, 192), (1024, 2880), (384, 104), (96, 64)])
 def test_transposed_quantise(shape):
     T, F = shape
     rng = np.random.default_rng(T + F)
@@ -214,6 +214,13 @@ def test_deosc_steps_bit_exact():
             assert np.array_equal(nibbles(host(out["codes_t"])[g]), nibbles(c_ref[g]).T)
     frozen = (st_ref >> 7).sum()
     assert frozen > 0                     # the boundary weights did oscillate and freeze
+
+
+def test_misaligned_rows_are_rejected():
+    x = torch.zeros((64, 100), dtype=torch.bfloat16, device="cuda")      # 200-byte rows
+    with pytest.raises(mxfp4.MXFP4Error) as e:
+        mxfp4.quantize(x, along_rows=True)
+    assert e.value.status == -3
 
 
 def test_bad_arguments_are_rejected_before_launch():
