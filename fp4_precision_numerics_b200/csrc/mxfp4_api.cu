@@ -191,9 +191,10 @@ mxfp4_status mxfp4_check_device_status(void* stream) {
     e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (v & mxfp4::kStatusTimeout)
-        return fail(MXFP4_ERR_DEVICE_TIMEOUT, "device wait timed out (status 0x%08x: roles %s%s%s%s)", v,
+        return fail(MXFP4_ERR_DEVICE_TIMEOUT, "device wait timed out (status 0x%08x: roles %s%s%s%s%s)", v,
                     (v & mxfp4::kRoleProducer) ? "producer " : "", (v & mxfp4::kRoleMma) ? "mma " : "",
-                    (v & mxfp4::kRoleEpilogue) ? "epilogue " : "", (v & mxfp4::kRoleTeardown) ? "teardown" : "");
+                    (v & mxfp4::kRoleEpilogue) ? "epilogue " : "", (v & mxfp4::kRoleScales) ? "scales " : "",
+                    (v & mxfp4::kRoleTeardown) ? "teardown" : "");
     return fail(MXFP4_ERR_DEVICE_BAD_INPUT, "device rejected group offsets (status 0x%08x)", v);
 }
 
@@ -322,6 +323,8 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
     if (num_groups <= 0 || !group_offsets || !A.codes || !A.scales_mma || !B.codes || !B.scales_mma || !out)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: null pointer or num_groups <= 0");
     if (M < 0 || N <= 0 || K < 0 || ldo < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad geometry");
+    if (num_groups > kMaxGroups)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: at most %d groups", kMaxGroups);
     if (K % 128 && op == MXFP4_GEMM_WGRAD)
         return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm(wgrad): total tokens must be a multiple of 128");
     if (K % 64) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: K %% 64 != 0");

@@ -196,8 +196,8 @@ typedef struct {
  *    D: [G, M, N], D_g = A[:, off[g]:off[g+1]] * B[:, off[g]:off[g+1]]^T,
  *    row stride ldo, group stride M*ldo; an empty group gives zeros.
  *  group_offsets: device int32 [G+1], non-decreasing, multiples of 128,
- *    group_offsets[0] = 0 (checked on the device; a bad group sets
- *    MXFP4_ERR_DEVICE_BAD_INPUT and its tiles are skipped).
+ *    group_offsets[0] = 0, G <= 1023.  Checked on the device: an invalid
+ *    array records MXFP4_ERR_DEVICE_BAD_INPUT and the call writes nothing.
  *  M_or_total: FPROP/DGRAD M (= off[G]); WGRAD: M.  K_or_total: FPROP/DGRAD
  *    K; WGRAD: off[G].  Tiles are 128 x 192 (both expert widths, 2880 and
  *    5760, are multiples of 192; other N are clipped at the edge),
