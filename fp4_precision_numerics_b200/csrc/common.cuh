@@ -39,22 +39,35 @@ struct Philox4 {
     uint32_t w[4];
 };
 
-__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3, uint32_t k0,
-                                                 uint32_t k1) {
+// The ten round keys of one Philox key, computed once per thread.
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+
+__device__ __forceinline__ PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
+    PhiloxKeys k;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        k.k0[r] = k0 + uint32_t(r) * 0x9E3779B9u;
+        k.k1[r] = k1 + uint32_t(r) * 0xBB67AE85u;
+    }
+    return k;
+}
+
+__device__ __forceinline__ Philox4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                                 const PhiloxKeys& k) {
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
         const uint32_t lo0 = 0xD2511F53u * c0;
         const uint32_t hi0 = __umulhi(0xD2511F53u, c0);
         const uint32_t lo1 = 0xCD9E8D57u * c2;
         const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2);
-        const uint32_t n0 = hi1 ^ c1 ^ k0;
-        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        const uint32_t n0 = hi1 ^ c1 ^ k.k0[round];
+        const uint32_t n2 = hi0 ^ c3 ^ k.k1[round];
         c0 = n0;
         c1 = lo1;
         c2 = n2;
         c3 = lo0;
-        k0 += 0x9E3779B9u;
-        k1 += 0xBB67AE85u;
     }
     Philox4 r;
     r.w[0] = c0;
@@ -82,26 +95,27 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
 // Stochastic rounding of v (already scaled into the block's range) onto the
 // E2M1 grid, returning a float that lies exactly on the grid (with v's
 // sign).  Rounds the magnitude up iff r16 * 2^-16 < f, f the position of
-// |v| between its neighbouring grid points; |v| >= 6 gives 6.
+// |v| between its neighbouring grid points; |v| >= 6 gives 6.  r6 = r16 << 6.
 //   |v| >= 1 : grid step is half the binade -> keep 1 mantissa bit; adding
 //              (2^22 - 1) - r16*2^6 to the bit pattern carries into bit 22
 //              exactly when the dropped 22 bits exceed r16*2^6.
 //   [.5, 1)  : step 0.5 = the binade -> keep 0 mantissa bits, same trick
 //              with 23 dropped bits and r16*2^7.
-//   [0, .5)  : result 0.5 iff r16 < |v| * 2^17 (exact float compare), else 0.
-__device__ __forceinline__ float e2m1_sr_value(float v, uint32_t r16) {
+//   [0, .5)  : 0.5 iff r16 < |v|*2^17, i.e. r16*2^6 < ceil(|v|*2^23); the
+//              ceiling comes exactly from adding 2^23 rounding upward.
+__device__ __forceinline__ float e2m1_sr_value(float v, uint32_t r6) {
     const uint32_t bits = __float_as_uint(v);
-    const uint32_t sign = bits & 0x80000000u;
     const uint32_t abits = bits & 0x7FFFFFFFu;
-    const float a = __uint_as_float(abits);
-    const uint32_t sh = abits < 0x3F800000u ? 23u : 22u;
-    const uint32_t mask = (1u << sh) - 1u;
-    const uint32_t rnd = mask - (r16 << (sh - 16u));
-    const float big = __uint_as_float((abits + rnd) & ~mask);
-    const float small = (__uint2float_rn(r16) < a * 131072.0f) ? 0.5f : 0.0f;
+    const bool ge1 = abits >= 0x3F800000u;
+    const uint32_t mask = ge1 ? 0x3FFFFFu : 0x7FFFFFu;
+    const uint32_t rs = ge1 ? r6 : (r6 << 1);
+    const float big = __uint_as_float((abits + (mask ^ rs)) & ~mask);
+    const uint32_t xi =
+        __float_as_uint(__fadd_ru(__fmul_rn(__uint_as_float(abits), 8388608.0f), 8388608.0f)) - 0x4B000000u;
+    const float small = r6 < xi ? 0.5f : 0.0f;
     float m = abits < 0x3F000000u ? small : big;
     m = fminf(m, 6.0f);
-    return __uint_as_float(__float_as_uint(m) | sign);
+    return __uint_as_float(__float_as_uint(m) | (bits & 0x80000000u));
 }
 
 // ---------------------------------------------------------------------------

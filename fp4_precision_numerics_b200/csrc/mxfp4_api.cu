@@ -79,7 +79,7 @@ unsigned grid_for(int64_t work, int threads) {
 // --- quantisation launchers --------------------------------------------------
 template <typename InT>
 mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
-    const int64_t work = qa.groups * qa.rows * (qa.cols / 16);
+    const int64_t work = qa.groups * qa.rows * (qa.cols / 32);
     const unsigned grid = grid_for(work, 256);
     if (rht && sr) mxfp4::quant1d_rows_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);
     else if (rht) mxfp4::quant1d_rows_kernel<InT, true, false><<<grid, 256, 0, st>>>(qa);
@@ -88,15 +88,37 @@ mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
     return check_launch("mxfp4_quantize(1d)");
 }
 
+bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box);
+
 template <typename InT>
 mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
-    const dim3 grid(unsigned((qa.rows + mxfp4::kTT - 1) / mxfp4::kTT), unsigned((qa.cols + mxfp4::kTF - 1) / mxfp4::kTF),
-                    unsigned(qa.groups));
-    if (rht && sr) mxfp4::quant1d_cols_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);
-    else if (rht) mxfp4::quant1d_cols_kernel<InT, true, false><<<grid, 256, 0, st>>>(qa);
-    else if (sr) mxfp4::quant1d_cols_kernel<InT, false, true><<<grid, 256, 0, st>>>(qa);
-    else mxfp4::quant1d_cols_kernel<InT, false, false><<<grid, 256, 0, st>>>(qa);
-    return check_launch("mxfp4_quantize(1d along rows)");
+    // input [groups][rows = T][cols = F] with row stride ld: box = 64 features x 128 tokens
+    CUtensorMap tm;
+    const uint64_t esz = sizeof(InT);
+    const uint64_t dims[3] = {uint64_t(qa.cols), uint64_t(qa.rows), uint64_t(qa.groups)};
+    const uint64_t strides[2] = {uint64_t(qa.ld) * esz, uint64_t(qa.ld) * esz * uint64_t(qa.rows)};
+    const uint32_t box[3] = {uint32_t(mxfp4::kTF), uint32_t(mxfp4::kTT), 1u};
+    if (!make_map_plain(&tm, sizeof(InT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                        qa.in, dims, strides, box))
+        return fail(MXFP4_ERR_CUDA, "mxfp4_quantize(along rows): tensor map encode failed");
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_quantize: cannot resolve the device status word");
+    const int64_t tiles = qa.groups * ((qa.rows + mxfp4::kTT - 1) / mxfp4::kTT) *
+                          ((qa.cols + mxfp4::kTF - 1) / mxfp4::kTF);
+    const int64_t cap = int64_t(num_sms()) * 4;
+    const unsigned grid = unsigned(tiles < cap ? tiles : cap);
+    const uint32_t smem = mxfp4::cols_smem_bytes<InT>();
+    auto go = [&](auto kern) -> mxfp4_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(MXFP4_ERR_CUDA, "mxfp4_quantize(along rows): shared-memory attribute");
+        kern<<<grid, 256, smem, st>>>(tm, qa, status);
+        return check_launch("mxfp4_quantize(1d along rows)");
+    };
+    if (rht && sr) return go(mxfp4::quant1d_cols_kernel<InT, true, true>);
+    if (rht) return go(mxfp4::quant1d_cols_kernel<InT, true, false>);
+    if (sr) return go(mxfp4::quant1d_cols_kernel<InT, false, true>);
+    return go(mxfp4::quant1d_cols_kernel<InT, false, false>);
 }
 
 template <typename InT, bool DEOSC>
@@ -156,6 +178,22 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
     for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
     return fn(m, dt, cuuint32_t(rank), const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t d[3], s[2];
+    cuuint32_t b[3], e[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+    }
+    for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+    return fn(m, dt, cuuint32_t(rank), const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

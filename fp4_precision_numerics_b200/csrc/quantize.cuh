@@ -111,8 +111,8 @@ __device__ __forceinline__ float amax16(const float (&x)[16]) {
 // Scale 16 values by 2^-E and round them to 8 bytes of packed codes.
 // `n0` is the SR element index of x[0] (multiple of 8).
 template <bool SR>
-__device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, uint32_t key0,
-                                         uint32_t key1, uint32_t offset) {
+__device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, const PhiloxKeys& keys,
+                                         uint32_t offset) {
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(x[i], inv_scale);
@@ -121,11 +121,12 @@ __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, 
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
             const uint64_t g = g0 + half;
-            const Philox4 r = philox4x32_10(uint32_t(g), uint32_t(g >> 32), offset, 0u, key0, key1);
+            const Philox4 r = philox4x32_10(uint32_t(g), uint32_t(g >> 32), offset, 0u, keys);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const uint32_t r16 = (r.w[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-                v[8 * half + j] = e2m1_sr_value(v[8 * half + j], r16);
+                const uint32_t wj = r.w[j >> 1];
+                const uint32_t r6 = (j & 1) ? ((wj >> 10) & 0x3FFFC0u) : ((wj << 6) & 0x3FFFC0u);
+                v[8 * half + j] = e2m1_sr_value(v[8 * half + j], r6);
             }
         }
     }
@@ -139,122 +140,147 @@ __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, 
 }
 
 // ---------------------------------------------------------------------------
-// 1D blocks along the last dim.  One thread per 16-element chunk; the two
-// threads of a 32-element block are adjacent lanes and combine their maxima
-// with one shuffle.  Output rows = input rows (groups back to back).
+// 1D blocks along the last dim.  One thread per 32-element block: two
+// 16-element RHT chunks in registers, the block maximum, scale, rounding,
+// and one 16-byte store of codes (consecutive threads write consecutive
+// blocks, so a warp's code stores are contiguous).  Output rows = input rows
+// (groups back to back).
 // ---------------------------------------------------------------------------
 template <typename InT, bool RHT, bool SR>
 __global__ void __launch_bounds__(256) quant1d_rows_kernel(QuantArgs a) {
     const int64_t C = a.cols;
-    const int64_t chunks_per_row = C >> 4;
-    const int64_t total_rows = a.groups * a.rows;
-    const int64_t total = total_rows * chunks_per_row;
     const int64_t S = C >> 5;
+    const int64_t total = a.groups * a.rows * S;
     const int64_t mma_group_bytes = mma_scale_bytes(a.rows, S);
     const InT* in = static_cast<const InT*>(a.in);
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    // Whole warps iterate together (the pair shuffle uses the full mask);
-    // `total` is even, so the two lanes of a block are valid together.
-    const int64_t first = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int lane = threadIdx.x & 31;
-    for (int64_t i = first; i - lane < total; i += stride) {
-        const bool valid = i < total;
-        const int64_t ic = valid ? i : total - 2 + (lane & 1);
-        const int64_t row = ic / chunks_per_row;
-        const int64_t col0 = (ic - row * chunks_per_row) << 4;
-        float x[16];
-        Loader<InT>::load16(in + row * a.ld + col0, x);
-        if constexpr (RHT) rht16(x, a.rht_signs);
-        float m = amax16(x);
-        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        if (!valid) continue;
-        const int sb = scale_byte_from_amax(m);
-        const uint2 q = quant16<SR>(x, inv_scale_from_byte(sb), uint64_t(row) * uint64_t(C) + uint64_t(col0),
-                                    a.sr_key0, a.sr_key1, a.sr_offset);
-        *reinterpret_cast<uint2*>(a.codes + row * (C >> 1) + (col0 >> 1)) = q;
-        if ((col0 & 16) == 0) {
-            const int64_t s = col0 >> 5;
-            if (a.scales) a.scales[row * S + s] = uint8_t(sb);
-            if (a.scales_mma) {
-                const int64_t g = row / a.rows, r = row - g * a.rows;
-                a.scales_mma[g * mma_group_bytes + mma_scale_offset(r, s, S)] = uint8_t(sb);
-            }
+    PhiloxKeys keys;
+    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t row = i / S;
+        const int64_t s = i - row * S;
+        const int64_t col0 = s << 5;
+        float x0[16], x1[16];
+        Loader<InT>::load16(in + row * a.ld + col0, x0);
+        Loader<InT>::load16(in + row * a.ld + col0 + 16, x1);
+        if constexpr (RHT) {
+            rht16(x0, a.rht_signs);
+            rht16(x1, a.rht_signs);
+        }
+        const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
+        const float inv = inv_scale_from_byte(sb);
+        const uint64_t n0 = uint64_t(row) * uint64_t(C) + uint64_t(col0);
+        const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
+        const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
+        *reinterpret_cast<uint4*>(a.codes + row * (C >> 1) + (col0 >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+        if (a.scales) a.scales[i] = uint8_t(sb);
+        if (a.scales_mma) {
+            const int64_t g = row / a.rows, r = row - g * a.rows;
+            a.scales_mma[g * mma_group_bytes + mma_scale_offset(r, s, S)] = uint8_t(sb);
         }
     }
 }
 
 // ---------------------------------------------------------------------------
 // 1D blocks along dim 0 (the token dim), output transposed: input [T, F]
-// (per group), output [F, T].  A CTA stages a 128-token x 64-feature tile in
-// shared memory with coalesced row loads; each thread then owns one
-// (feature, 32-token block): RHT on its two chunks, amax, scale, rounding,
-// and one 16-byte store of codes into output row `feature`.
+// (per group), output [F, T].  Persistent CTAs walk 128-token x 64-feature
+// tiles; a 3-deep ring of shared-memory buffers is filled by TMA (zero fill
+// at the ragged edges), so the next tiles stream in while the current one
+// is quantised.  Each thread owns one (feature, 32-token block): RHT on its
+// two 16-token chunks, amax, scale, rounding, one 16-byte store of codes.
 // ---------------------------------------------------------------------------
-constexpr int kTT = 128;  // tokens per tile
-constexpr int kTF = 64;   // features per tile
+constexpr int kTT = 128;    // tokens per tile
+constexpr int kTF = 64;     // features per tile
+constexpr int kColsRing = 3;
+
+template <typename InT>
+__host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(kTT * kTF * sizeof(InT)); }
+
+template <typename InT>
+__host__ __device__ constexpr uint32_t cols_smem_bytes() { return kColsRing * cols_tile_bytes<InT>() + 64 + 128; }
 
 template <typename InT, bool RHT, bool SR>
-__global__ void __launch_bounds__(256) quant1d_cols_kernel(QuantArgs a) {
-    __shared__ __align__(16) InT tile[kTT][kTF + 16 / sizeof(InT)];
+__global__ void __launch_bounds__(256) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
+                                                           uint32_t* status) {
+    extern __shared__ uint8_t cols_smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(cols_smem_raw) + 127) & ~uintptr_t(127));
+    constexpr uint32_t kTile = cols_tile_bytes<InT>();
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + kColsRing * kTile);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kColsRing * kTile + 8 * kColsRing);
     const int64_t T = a.rows, F = a.cols;
-    const int64_t g = blockIdx.z;
-    const int64_t t0 = int64_t(blockIdx.x) * kTT;
-    const int64_t f0 = int64_t(blockIdx.y) * kTF;
-    const InT* in = static_cast<const InT*>(a.in) + g * T * a.ld;
-    // stage: 16-byte vectors along the feature dim
-    constexpr int kVec = 16 / sizeof(InT);
-    constexpr int kVecPerRow = kTF / kVec;
-    for (int idx = threadIdx.x; idx < kTT * kVecPerRow; idx += blockDim.x) {
-        const int tr = idx / kVecPerRow;
-        const int fv = (idx - tr * kVecPerRow) * kVec;
-        const int64_t t = t0 + tr, f = f0 + fv;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < T) {
-            if (f + kVec <= F) {
-                v = __ldg(reinterpret_cast<const uint4*>(in + t * a.ld + f));
-            } else {
-                InT tmp[kVec];
-#pragma unroll
-                for (int k = 0; k < kVec; ++k) tmp[k] = (f + k < F) ? in[t * a.ld + f + k] : InT(0);
-                v = *reinterpret_cast<const uint4*>(tmp);
-            }
+    const int64_t ntt = (T + kTT - 1) / kTT, ntf = (F + kTF - 1) / kTF;
+    const int64_t ntiles = a.groups * ntt * ntf;
+    const int64_t first = blockIdx.x;
+    const int64_t mine = first < ntiles ? (ntiles - first + gridDim.x - 1) / gridDim.x : 0;
+    auto tile_coords = [&](int64_t i, int64_t& g, int64_t& t0, int64_t& f0) {
+        const int64_t t = first + i * gridDim.x;
+        g = t / (ntt * ntf);
+        const int64_t r = t - g * ntt * ntf;
+        t0 = (r / ntf) * kTT;
+        f0 = (r - (r / ntf) * ntf) * kTF;
+    };
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < kColsRing; ++b) mbar_init(&full[b], 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&tm_in);
+        for (int64_t i = 0; i < mine && i < kColsRing; ++i) {
+            int64_t g, t0, f0;
+            tile_coords(i, g, t0, f0);
+            mbar_arrive_expect_tx(&full[i], kTile);
+            tma_load_3d(smem + i * kTile, &tm_in, &full[i], int32_t(f0), int32_t(t0), int32_t(g));
         }
-        *reinterpret_cast<uint4*>(&tile[tr][fv]) = v;
     }
     __syncthreads();
-    // one (feature, block) per thread: 64 features x 4 blocks
+    PhiloxKeys keys;
+    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
     const int fl = threadIdx.x & 63;
     const int blk = threadIdx.x >> 6;
-    const int64_t f = f0 + fl;
-    const int64_t tb = t0 + blk * 32;
-    if (f >= F || tb >= T) return;
-    float x0[16], x1[16];
+    const int64_t S = T >> 5;
+    for (int64_t i = 0; i < mine; ++i) {
+        const int b = int(i % kColsRing);
+        const uint32_t phase = uint32_t(i / kColsRing) & 1u;
+        const bool got = mbar_wait_bounded(&full[b], phase, abort_flag, status, kRoleProducer);
+        int64_t g, t0, f0;
+        tile_coords(i, g, t0, f0);
+        const int64_t f = f0 + fl;
+        const int64_t tb = t0 + blk * 32;
+        if (got && f < F && tb < T) {
+            const InT* tile = reinterpret_cast<const InT*>(smem + b * kTile);   // [kTT][kTF], dense
+            float x0[16], x1[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        if constexpr (sizeof(InT) == 2) {
-            x0[k] = __uint_as_float(uint32_t(tile[blk * 32 + k][fl]) << 16);
-            x1[k] = __uint_as_float(uint32_t(tile[blk * 32 + 16 + k][fl]) << 16);
-        } else {
-            x0[k] = tile[blk * 32 + k][fl];
-            x1[k] = tile[blk * 32 + 16 + k][fl];
+            for (int k = 0; k < 16; ++k) {
+                if constexpr (sizeof(InT) == 2) {
+                    x0[k] = __uint_as_float(uint32_t(tile[(blk * 32 + k) * kTF + fl]) << 16);
+                    x1[k] = __uint_as_float(uint32_t(tile[(blk * 32 + 16 + k) * kTF + fl]) << 16);
+                } else {
+                    x0[k] = tile[(blk * 32 + k) * kTF + fl];
+                    x1[k] = tile[(blk * 32 + 16 + k) * kTF + fl];
+                }
+            }
+            if constexpr (RHT) {
+                rht16(x0, a.rht_signs);
+                rht16(x1, a.rht_signs);
+            }
+            const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
+            const float inv = inv_scale_from_byte(sb);
+            const int64_t orow = g * F + f;  // output row (groups back to back)
+            const uint64_t n0 = uint64_t(orow) * uint64_t(T) + uint64_t(tb);
+            const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
+            const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
+            *reinterpret_cast<uint4*>(a.codes + orow * (T >> 1) + (tb >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+            const int64_t s = tb >> 5;
+            if (a.scales) a.scales[orow * S + s] = uint8_t(sb);
+            if (a.scales_mma) a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f, s, S)] = uint8_t(sb);
+        }
+        __syncthreads();  // buffer b fully read: refill it with tile i + kColsRing
+        if (threadIdx.x == 0 && i + kColsRing < mine) {
+            int64_t g2, t2, f2;
+            tile_coords(i + kColsRing, g2, t2, f2);
+            mbar_arrive_expect_tx(&full[b], kTile);
+            tma_load_3d(smem + b * kTile, &tm_in, &full[b], int32_t(f2), int32_t(t2), int32_t(g2));
         }
     }
-    if constexpr (RHT) {
-        rht16(x0, a.rht_signs);
-        rht16(x1, a.rht_signs);
-    }
-    const float m = fmaxf(amax16(x0), amax16(x1));
-    const int sb = scale_byte_from_amax(m);
-    const float inv = inv_scale_from_byte(sb);
-    const int64_t orow = g * F + f;  // output row (groups back to back)
-    const uint64_t n0 = uint64_t(orow) * uint64_t(T) + uint64_t(tb);
-    const uint2 q0 = quant16<SR>(x0, inv, n0, a.sr_key0, a.sr_key1, a.sr_offset);
-    const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, a.sr_key0, a.sr_key1, a.sr_offset);
-    *reinterpret_cast<uint4*>(a.codes + orow * (T >> 1) + (tb >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-    const int64_t S = T >> 5;
-    const int64_t s = tb >> 5;
-    if (a.scales) a.scales[orow * S + s] = uint8_t(sb);
-    if (a.scales_mma) a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f, s, S)] = uint8_t(sb);
 }
 
 // ---------------------------------------------------------------------------
@@ -291,43 +317,54 @@ __global__ void __launch_bounds__(256) quant2d_kernel(QuantArgs a) {
     const int sb = scale_byte_from_amax(m);
     const float inv = inv_scale_from_byte(sb);
     const uint64_t n0 = (uint64_t(g) * uint64_t(R) + uint64_t(r)) * uint64_t(C) + uint64_t(c0);
-    uint2 q0 = quant16<SR>(x0, inv, n0, a.sr_key0, a.sr_key1, a.sr_offset);
-    uint2 q1 = quant16<SR>(x1, inv, n0 + 16, a.sr_key0, a.sr_key1, a.sr_offset);
+    PhiloxKeys keys;
+    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
+    uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
+    uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
     uint32_t w[4] = {q0.x, q0.y, q1.x, q1.y};  // 32 codes of row r, nibble k = element k
     const int64_t widx = (g * R + r) * C + c0;  // weight index of element 0 of this row
     if constexpr (DEOSC) {
-        uint4 st0 = *reinterpret_cast<const uint4*>(a.state + widx);
-        uint4 st1 = *reinterpret_cast<const uint4*>(a.state + widx + 16);
+        // Byte-parallel state update: four weights per 32-bit word.  The
+        // codes of 8 weights (one nibble each) are spread to two words of
+        // 4 bytes, updated with carry-free byte arithmetic, and packed back.
+        const uint4 st0 = *reinterpret_cast<const uint4*>(a.state + widx);
+        const uint4 st1 = *reinterpret_cast<const uint4*>(a.state + widx + 16);
         uint32_t s[8] = {st0.x, st0.y, st0.z, st0.w, st1.x, st1.y, st1.z, st1.w};
         const bool reset = a.step > 0 && a.reset_period > 0 && (a.step % a.reset_period) == 0;
+        const uint32_t thr_bias = (0x80u - a.flip_threshold) * 0x01010101u;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const uint32_t q = (w[k >> 3] >> (4 * (k & 7))) & 0xFu;
-            uint32_t st = (s[k >> 2] >> (8 * (k & 3))) & 0xFFu;
-            uint32_t outc;
-            if (a.step == 0) {
-                st = q;
-                outc = q;
-            } else {
-                uint32_t prev = st & 0xFu, cnt = (st >> 4) & 7u, frz = st >> 7;
+        for (int m = 0; m < 4; ++m) {
+            const uint32_t ev = w[m] & 0x0F0F0F0Fu;          // codes 8m+0, +2, +4, +6
+            const uint32_t od = (w[m] >> 4) & 0x0F0F0F0Fu;   // codes 8m+1, +3, +5, +7
+            uint32_t q[2] = {__byte_perm(ev, od, 0x5140), __byte_perm(ev, od, 0x7362)};
+            uint32_t o[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t S = s[2 * m + h], Q = q[h];
+                if (a.step == 0) {
+                    s[2 * m + h] = Q;
+                    o[h] = Q;
+                    continue;
+                }
+                const uint32_t prev = S & 0x0F0F0F0Fu;
+                uint32_t cnt = (S >> 4) & 0x07070707u;
+                uint32_t frz = S & 0x80808080u;
                 if (reset) {
-                    cnt = 0;
-                    frz = 0;
+                    cnt = 0u;
+                    frz = 0u;
                 }
-                if (frz) {
-                    outc = prev;
-                } else {
-                    if (q != prev) {
-                        cnt = cnt < 7u ? cnt + 1u : 7u;
-                        prev = q;
-                        if (cnt >= a.flip_threshold) frz = 1;
-                    }
-                    outc = q;
-                }
-                st = prev | (cnt << 4) | (frz << 7);
+                const uint32_t ne = ((Q ^ prev) + 0x7F7F7F7Fu) & 0x80808080u;  // 0x80 where q != prev
+                const uint32_t upd = ne & ~frz;                                 // 0x80 where the weight flips
+                uint32_t c2 = cnt + (upd >> 7);
+                c2 -= (c2 >> 3) & 0x01010101u;                                  // saturate 8 -> 7
+                const uint32_t updm = (upd >> 7) * 0xFFu;
+                const uint32_t frzm = (frz >> 7) * 0xFFu;
+                const uint32_t prev2 = (Q & updm) | (prev & ~updm);
+                const uint32_t frz2 = frz | (upd & ((c2 + thr_bias) & 0x80808080u));
+                s[2 * m + h] = prev2 | (c2 << 4) | frz2;
+                o[h] = (prev & frzm) | (Q & ~frzm);                             // frozen: stored code
             }
-            s[k >> 2] = (s[k >> 2] & ~(0xFFu << (8 * (k & 3)))) | (st << (8 * (k & 3)));
-            w[k >> 3] = (w[k >> 3] & ~(0xFu << (4 * (k & 7)))) | (outc << (4 * (k & 7)));
+            w[m] = __byte_perm(o[0], o[1], 0x6420) | (__byte_perm(o[0], o[1], 0x7531) << 4);
         }
         *reinterpret_cast<uint4*>(a.state + widx) = make_uint4(s[0], s[1], s[2], s[3]);
         *reinterpret_cast<uint4*>(a.state + widx + 16) = make_uint4(s[4], s[5], s[6], s[7]);
