@@ -181,15 +181,17 @@ def quantize_1d(x: np.ndarray, rht_d: int = 0, rht_seed: int = 0, sr: bool = Fal
 
 
 def quantize_1d_transposed(x: np.ndarray, rht_d: int = 0, rht_seed: int = 0, sr: bool = False,
-                           sr_seed: int = 0, sr_offset: int = 0):
+                           sr_seed: int = 0, sr_offset: int = 0, col0: int = 0):
     """1x32 blocks along dim 0; output in the transposed layout
-    (codes [C, R/2], scales [C, R/32])."""
+    (codes [C, R/2], scales [C, R/32]).  `col0` is the global index of x's
+    first column (= first output row), so a column slice draws the same SR
+    bits as the whole tensor."""
     x, dt = _input(x)
     rows, cols = x.shape
     codes = np.zeros((cols, rows // 2), dtype=np.uint8)
     scales = np.zeros((cols, rows // 32), dtype=np.uint8)
     lib().oracle_quantize_1d_transposed(_ptr(x), dt, rows, cols, cols, rht_d, rht_seed, int(sr), sr_seed,
-                                        sr_offset, 0, _ptr(codes), _ptr(scales))
+                                        sr_offset, col0, _ptr(codes), _ptr(scales))
     return codes, scales
 
 
