@@ -2,6 +2,7 @@
 // argument validation, tensor-map encoding and kernel launches on the
 // caller's stream.  No allocation, no exceptions across the boundary.
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -10,6 +11,7 @@
 #include "../../include/mxfp4.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -42,6 +44,37 @@ int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     return n;
+}
+
+// Clusters of two CTAs of the pair GEMM that can be resident at once (one
+// CTA per SM; an SM left without a partner in its GPC stays idle).
+int pair_clusters() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms() / 2;
+    if (cached[dev] > 0) return cached[dev];
+    int n = 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * unsigned(num_sms() / 2), 1, 1);
+    cfg.blockDim = dim3(mxfp4::gemm2::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = mxfp4::gemm2::kSmemBytes;
+    if (cudaOccupancyMaxActiveClusters(&n, mxfp4::gemm2::grouped_gemm_2sm_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms() / 2;
+    }
+    cached[dev] = n;
+    return n;
+}
+
+// The one-CTA GEMM serves more than gemm2::kMaxGroups groups, and is also
+// chosen for every call when MXFP4_GEMM_CTA_PAIRS=0 is set in the
+// environment (for side-by-side measurement).
+bool pairs_enabled() {
+    static const bool on = [] {
+        const char* v = getenv("MXFP4_GEMM_CTA_PAIRS");
+        return !(v && v[0] == '0');
+    }();
+    return on;
 }
 
 uint32_t* status_word() {
@@ -403,6 +436,8 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
     a.total_tiles = a.mode == 0 ? int64_t(a.m_tiles) * a.n_tiles : int64_t(num_groups) * a.m_tiles * a.n_tiles;
     a.status = status;
 
+    const bool pair = pairs_enabled() && num_groups <= mxfp4::gemm2::kMaxGroups;
+    const uint32_t b_rows = pair ? uint32_t(mxfp4::gemm2::BNH) : uint32_t(BN);
     CUtensorMap tmA, tmB, tmD;
     const uint64_t kb = uint64_t(K / 2);
     {
@@ -415,7 +450,7 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
     if (a.mode == 0) {
         const uint64_t dims[3] = {kb, uint64_t(N), uint64_t(num_groups)};
         const uint64_t str[2] = {kb, kb * uint64_t(N)};
-        const uint32_t box[3] = {128, BN, 1};
+        const uint32_t box[3] = {128, b_rows, 1};
         if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, B.codes, dims, str, box))
             return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
         const uint64_t ddims[2] = {uint64_t(N), uint64_t(M)};
@@ -426,7 +461,7 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
     } else {
         const uint64_t dims[2] = {kb, uint64_t(N)};
         const uint64_t str[1] = {kb};
-        const uint32_t box[2] = {128, BN};
+        const uint32_t box[2] = {128, b_rows};
         if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, B.codes, dims, str, box))
             return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
         const uint64_t ddims[3] = {uint64_t(N), uint64_t(M), uint64_t(num_groups)};
@@ -434,6 +469,22 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
         const uint32_t dbox[3] = {32, 32, 1};
         if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, ddims, dstr, dbox))
             return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
+    }
+    if (pair) {
+        namespace g2 = mxfp4::gemm2;
+        if (cudaFuncSetAttribute(g2::grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 g2::kSmemBytes) != cudaSuccess)
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
+        // upper bound on the units (group, m-tile pair, n-tile): the exact
+        // count depends on the device-side offsets
+        const int64_t units = a.mode == 0 ? (int64_t(a.m_tiles) / 2 + num_groups) * a.n_tiles
+                                          : int64_t(num_groups) * ((a.m_tiles + 1) / 2) * a.n_tiles;
+        if (units == 0) return ok();
+        const int64_t clusters = pair_clusters();
+        const unsigned grid = 2u * unsigned(units < clusters ? units : clusters);
+        g2::grouped_gemm_2sm_kernel<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
+            tmA, tmB, tmD, a);
+        return check_launch("mxfp4_grouped_gemm");
     }
     if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
         cudaSuccess)
