@@ -157,14 +157,15 @@ mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
 template <typename InT, bool DEOSC>
 mxfp4_status launch_2d(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
     const int64_t nblocks = qa.groups * (qa.rows / 32) * (qa.cols / 32);
-    const unsigned grid = unsigned((nblocks + 7) / 8);
+    constexpr int kThreads2d = 256;   // warps of a CTA take neighbouring blocks of a block row
+    const unsigned grid = unsigned((nblocks + kThreads2d / 32 - 1) / (kThreads2d / 32));
     if constexpr (DEOSC) {
-        mxfp4::quant2d_kernel<InT, false, false, true><<<grid, 256, 0, st>>>(qa);
+        mxfp4::quant2d_kernel<InT, false, false, true><<<grid, kThreads2d, 0, st>>>(qa);
     } else {
-        if (rht && sr) mxfp4::quant2d_kernel<InT, true, true, false><<<grid, 256, 0, st>>>(qa);
-        else if (rht) mxfp4::quant2d_kernel<InT, true, false, false><<<grid, 256, 0, st>>>(qa);
-        else if (sr) mxfp4::quant2d_kernel<InT, false, true, false><<<grid, 256, 0, st>>>(qa);
-        else mxfp4::quant2d_kernel<InT, false, false, false><<<grid, 256, 0, st>>>(qa);
+        if (rht && sr) mxfp4::quant2d_kernel<InT, true, true, false><<<grid, kThreads2d, 0, st>>>(qa);
+        else if (rht) mxfp4::quant2d_kernel<InT, true, false, false><<<grid, kThreads2d, 0, st>>>(qa);
+        else if (sr) mxfp4::quant2d_kernel<InT, false, true, false><<<grid, kThreads2d, 0, st>>>(qa);
+        else mxfp4::quant2d_kernel<InT, false, false, false><<<grid, kThreads2d, 0, st>>>(qa);
     }
     return check_launch(DEOSC ? "mxfp4_deosc_update" : "mxfp4_quantize(2d)");
 }

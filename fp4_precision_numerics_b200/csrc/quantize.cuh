@@ -285,28 +285,70 @@ __global__ void __launch_bounds__(256) quant1d_cols_kernel(const __grid_constant
 
 // ---------------------------------------------------------------------------
 // 2D 32x32 blocks (weights), optionally with the de-oscillation update.
-// One warp per block; lane l owns row l of the block (32 elements).  The
-// codes of the transpose are produced through a padded shared-memory copy
-// of the block's 32x32 code bytes.
+// One warp per block; lane l owns row l of the block (32 elements), and the
+// warps of a CTA take neighbouring blocks of a block row, so the row
+// segments they read together share DRAM pages.  The codes of the transpose
+// come from a register transpose across the warp (five shuffle stages).
 // ---------------------------------------------------------------------------
+// Transpose a 32 x 32 matrix of 4-bit codes held one row per lane (nibble k
+// of word m of lane r = element (r, 8m + k)) so that lane c ends up with
+// column c in the same format.  Five butterfly stages exchange blocks of 16,
+// 8, 4, 2 and 1 codes with the lane at distance 16, 8, 4, 2, 1.
+__device__ __forceinline__ void transpose32x32_nibbles(uint32_t (&w)[4], int lane) {
+    constexpr uint32_t kAll = 0xFFFFFFFFu;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {   // 16 codes: words (j) <-> (j + 2)
+        const bool up = lane & 16;
+        const uint32_t r = __shfl_xor_sync(kAll, up ? w[j] : w[j + 2], 16);
+        if (up) w[j] = r;
+        else w[j + 2] = r;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {   // 8 codes: words (j) <-> (j + 1)
+        const bool up = lane & 8;
+        const uint32_t r = __shfl_xor_sync(kAll, up ? w[j] : w[j + 1], 8);
+        if (up) w[j] = r;
+        else w[j + 1] = r;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {   // 4 codes: 16-bit halves, two words per shuffle
+        const uint32_t a = w[j], b = w[j + 1];
+        const bool up = lane & 4;
+        const uint32_t r = __shfl_xor_sync(kAll, up ? __byte_perm(a, b, 0x5410) : __byte_perm(a, b, 0x7632), 4);
+        w[j] = up ? __byte_perm(a, r, 0x3254) : __byte_perm(a, r, 0x5410);
+        w[j + 1] = up ? __byte_perm(b, r, 0x3276) : __byte_perm(b, r, 0x7610);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {   // 2 codes: bytes
+        const uint32_t a = w[j], b = w[j + 1];
+        const bool up = lane & 2;
+        const uint32_t r = __shfl_xor_sync(kAll, up ? __byte_perm(a, b, 0x6420) : __byte_perm(a, b, 0x7531), 2);
+        w[j] = up ? __byte_perm(a, r, 0x3514) : __byte_perm(a, r, 0x5240);
+        w[j + 1] = up ? __byte_perm(b, r, 0x3716) : __byte_perm(b, r, 0x7260);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {   // 1 code: nibbles inside each byte
+        const uint32_t a = w[j], b = w[j + 1];
+        const bool up = lane & 1;
+        // the low (up) or high (!up) nibble of every byte, four per 16 bits
+        const uint32_t ta = up ? (a & 0x0F0F0F0Fu) : ((a >> 4) & 0x0F0F0F0Fu);
+        const uint32_t tb = up ? (b & 0x0F0F0F0Fu) : ((b >> 4) & 0x0F0F0F0Fu);
+        const uint32_t r = __shfl_xor_sync(kAll, __byte_perm(ta | (ta >> 4), tb | (tb >> 4), 0x6420), 1);
+        const uint32_t va = __byte_perm(r, 0u, 0x1100), vb = __byte_perm(r, 0u, 0x3322);
+        const uint32_t sa = (va & 0x000F000Fu) | ((va >> 4) & 0x0F000F00u);   // nibble k -> low nibble of byte k
+        const uint32_t sb = (vb & 0x000F000Fu) | ((vb >> 4) & 0x0F000F00u);
+        w[j] = up ? ((a & 0xF0F0F0F0u) | sa) : ((a & 0x0F0F0F0Fu) | (sa << 4));
+        w[j + 1] = up ? ((b & 0xF0F0F0F0u) | sb) : ((b & 0x0F0F0F0Fu) | (sb << 4));
+    }
+}
+
 template <typename InT, bool RHT, bool SR, bool DEOSC>
-__global__ void __launch_bounds__(256) quant2d_kernel(QuantArgs a) {
-    __shared__ uint32_t tcodes[8][32 * 9];  // per warp: 32 rows x 36 bytes
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int64_t bi, int64_t bj, int lane,
+                                              float (&x0)[16], float (&x1)[16], uint32_t (&s)[8]) {
     const int64_t R = a.rows, C = a.cols;
     const int64_t nbr = R >> 5, nbc = C >> 5;
-    const int64_t nblocks = a.groups * nbr * nbc;
-    const int64_t bid = int64_t(blockIdx.x) * 8 + warp;
-    if (bid >= nblocks) return;
-    const int64_t g = bid / (nbr * nbc);
-    const int64_t rem = bid - g * nbr * nbc;
-    const int64_t bi = rem / nbc, bj = rem - bi * nbc;
     const int64_t r = bi * 32 + lane;
     const int64_t c0 = bj * 32;
-    const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
-    float x0[16], x1[16];
-    Loader<InT>::load16(in + r * a.ld + c0, x0);
-    Loader<InT>::load16(in + r * a.ld + c0 + 16, x1);
     if constexpr (RHT) {
         rht16(x0, a.rht_signs);
         rht16(x1, a.rht_signs);
@@ -327,9 +369,6 @@ __global__ void __launch_bounds__(256) quant2d_kernel(QuantArgs a) {
         // Byte-parallel state update: four weights per 32-bit word.  The
         // codes of 8 weights (one nibble each) are spread to two words of
         // 4 bytes, updated with carry-free byte arithmetic, and packed back.
-        const uint4 st0 = *reinterpret_cast<const uint4*>(a.state + widx);
-        const uint4 st1 = *reinterpret_cast<const uint4*>(a.state + widx + 16);
-        uint32_t s[8] = {st0.x, st0.y, st0.z, st0.w, st1.x, st1.y, st1.z, st1.w};
         const bool reset = a.step > 0 && a.reset_period > 0 && (a.step % a.reset_period) == 0;
         const uint32_t thr_bias = (0x80u - a.flip_threshold) * 0x01010101u;
 #pragma unroll
@@ -374,25 +413,42 @@ __global__ void __launch_bounds__(256) quant2d_kernel(QuantArgs a) {
     if (a.scales && lane == 0) a.scales[g * nbr * nbc + bi * nbc + bj] = uint8_t(sb);
     if (a.scales_mma) a.scales_mma[g * mma_scale_bytes(R, S) + mma_scale_offset(r, bj, S)] = uint8_t(sb);
     if (a.codes_t) {
-        // byte k of row `lane` = code of element k (0..31), row pitch 36 bytes
-        uint32_t* t = tcodes[warp];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t src = w[j >> 1] >> (16 * (j & 1));  // codes 4j..4j+3
-            t[lane * 9 + j] = (src & 0xFu) | (((src >> 4) & 0xFu) << 8) | (((src >> 8) & 0xFu) << 16) |
-                              (((src >> 12) & 0xFu) << 24);
-        }
-        __syncwarp();
-        const uint8_t* tb = reinterpret_cast<const uint8_t*>(t);
-        uint32_t o[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i >> 3] |= uint32_t(tb[i * 36 + lane]) << (4 * (i & 7));
+        uint32_t o[4] = {w[0], w[1], w[2], w[3]};
+        transpose32x32_nibbles(o, lane);
         // row (c0 + lane) of W^T, columns r0..r0+31 of it are rows of this block
         const int64_t tr = g * C + c0 + lane;
         *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + (bi * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
         if (a.scales_mma_t)
             a.scales_mma_t[g * mma_scale_bytes(C, nbr) + mma_scale_offset(c0 + lane, bi, nbr)] = uint8_t(sb);
     }
+}
+
+template <typename InT, bool RHT, bool SR, bool DEOSC>
+__global__ void __launch_bounds__(1024) quant2d_kernel(QuantArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t R = a.rows, C = a.cols;
+    const int64_t nbr = R >> 5, nbc = C >> 5;
+    const int64_t nblocks = a.groups * nbr * nbc;
+    const int64_t bid = int64_t(blockIdx.x) * (blockDim.x >> 5) + warp;
+    if (bid >= nblocks) return;
+    const int64_t g = bid / (nbr * nbc);
+    const int64_t rem = bid - g * nbr * nbc;
+    const int64_t bi = rem / nbc, bj = rem - bi * nbc;
+    const int64_t r = bi * 32 + lane;
+    const int64_t c0 = bj * 32;
+    const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
+    float x0[16], x1[16];
+    Loader<InT>::load16(in + r * a.ld + c0, x0);
+    Loader<InT>::load16(in + r * a.ld + c0 + 16, x1);
+    uint32_t s[8];
+    if constexpr (DEOSC) {
+        const int64_t widx = (g * R + r) * C + c0;
+        const uint4 st0 = *reinterpret_cast<const uint4*>(a.state + widx);
+        const uint4 st1 = *reinterpret_cast<const uint4*>(a.state + widx + 16);
+        s[0] = st0.x; s[1] = st0.y; s[2] = st0.z; s[3] = st0.w;
+        s[4] = st1.x; s[5] = st1.y; s[6] = st1.z; s[7] = st1.w;
+    }
+    quant2d_block<InT, RHT, SR, DEOSC>(a, g, bi, bj, lane, x0, x1, s);
 }
 
 // ---------------------------------------------------------------------------
