@@ -157,8 +157,8 @@ mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
 template <typename InT, bool DEOSC>
 mxfp4_status launch_2d(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
     const int64_t nblocks = qa.groups * (qa.rows / 32) * (qa.cols / 32);
-    constexpr int kThreads2d = 256;   // warps of a CTA take neighbouring blocks of a block row
-    const unsigned grid = unsigned((nblocks + kThreads2d / 32 - 1) / (kThreads2d / 32));
+    constexpr int kThreads2d = mxfp4::kQ2dWarps * 32;   // warps of a CTA take neighbouring blocks of a block row
+    const unsigned grid = unsigned((nblocks + mxfp4::kQ2dWarps - 1) / mxfp4::kQ2dWarps);
     if constexpr (DEOSC) {
         mxfp4::quant2d_kernel<InT, false, false, true><<<grid, kThreads2d, 0, st>>>(qa);
     } else {

@@ -423,30 +423,61 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
     }
 }
 
+constexpr int kQ2dWarps = 8;   // warps (blocks) per CTA
+
 template <typename InT, bool RHT, bool SR, bool DEOSC>
-__global__ void __launch_bounds__(1024) quant2d_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_kernel(QuantArgs a) {
+    // Per warp: the block as 32 rows x 8 chunks of 4 binary32 (chunk c of row
+    // r at slot c ^ (r & 7)), and its 32 x 32 state bytes (word c of row r at
+    // slot c ^ ((r >> 2) & 7)); both swizzles keep the row-of-4-rows writes
+    // and the row-per-lane reads free of bank conflicts.
+    __shared__ float4 xs[kQ2dWarps][32 * 8];
+    __shared__ uint32_t ss[kQ2dWarps][DEOSC ? 32 * 8 : 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t R = a.rows, C = a.cols;
     const int64_t nbr = R >> 5, nbc = C >> 5;
     const int64_t nblocks = a.groups * nbr * nbc;
-    const int64_t bid = int64_t(blockIdx.x) * (blockDim.x >> 5) + warp;
+    const int64_t bid = int64_t(blockIdx.x) * kQ2dWarps + warp;
     if (bid >= nblocks) return;
     const int64_t g = bid / (nbr * nbc);
     const int64_t rem = bid - g * nbr * nbc;
     const int64_t bi = rem / nbc, bj = rem - bi * nbc;
-    const int64_t r = bi * 32 + lane;
     const int64_t c0 = bj * 32;
     const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
+    // Coalesced loads: instruction k covers rows 4k..4k+3 of the block, eight
+    // lanes per row (lane = 8 q + c: row 4k + q, elements 4c..4c+3).  One warp
+    // instruction touching 32 rows at once (a row per lane) reads DRAM at
+    // about two thirds of this rate.
+    const int q = lane >> 3, c = lane & 7;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int rr = 4 * k + q;
+        const InT* src = in + (bi * 32 + rr) * a.ld + c0 + 4 * c;
+        float4 v;
+        if constexpr (sizeof(InT) == 4) {
+            v = __ldg(reinterpret_cast<const float4*>(src));
+        } else {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
+            v = make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                            __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+        }
+        xs[warp][rr * 8 + (c ^ (rr & 7))] = v;
+        if constexpr (DEOSC)
+            ss[warp][rr * 8 + (c ^ k)] =
+                __ldg(reinterpret_cast<const uint32_t*>(a.state + (g * R + bi * 32 + rr) * C + c0 + 4 * c));
+    }
+    __syncwarp();
     float x0[16], x1[16];
-    Loader<InT>::load16(in + r * a.ld + c0, x0);
-    Loader<InT>::load16(in + r * a.ld + c0 + 16, x1);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float4 v = xs[warp][lane * 8 + (j ^ (lane & 7))];
+        float* dst = j < 4 ? &x0[4 * j] : &x1[4 * (j - 4)];
+        dst[0] = v.x; dst[1] = v.y; dst[2] = v.z; dst[3] = v.w;
+    }
     uint32_t s[8];
     if constexpr (DEOSC) {
-        const int64_t widx = (g * R + r) * C + c0;
-        const uint4 st0 = *reinterpret_cast<const uint4*>(a.state + widx);
-        const uint4 st1 = *reinterpret_cast<const uint4*>(a.state + widx + 16);
-        s[0] = st0.x; s[1] = st0.y; s[2] = st0.z; s[3] = st0.w;
-        s[4] = st1.x; s[5] = st1.y; s[6] = st1.z; s[7] = st1.w;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j] = ss[warp][lane * 8 + (j ^ ((lane >> 2) & 7))];
     }
     quant2d_block<InT, RHT, SR, DEOSC>(a, g, bi, bj, lane, x0, x1, s);
 }
