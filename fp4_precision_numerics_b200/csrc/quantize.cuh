@@ -109,33 +109,32 @@ __device__ __forceinline__ float amax16(const float (&x)[16]) {
 }
 
 // Scale 16 values by 2^-E and round them to 8 bytes of packed codes.
-// `n0` is the SR element index of x[0] (multiple of 8).
+// `n0` is the SR element index of x[0] (a multiple of 16): one Philox call
+// covers the 16 elements, word j the four elements 4j..4j+3, consumed by the
+// four-element stochastic-rounding conversion (see e2m1x4_sr).
 template <bool SR>
 __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, const PhiloxKeys& keys,
                                          uint32_t offset) {
     float v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(x[i], inv_scale);
-    if constexpr (SR) {
-        const uint64_t g0 = n0 >> 3;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const uint64_t g = g0 + half;
-            const Philox4 r = philox4x32_10(uint32_t(g), uint32_t(g >> 32), offset, 0u, keys);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t wj = r.w[j >> 1];
-                const uint32_t r6 = (j & 1) ? ((wj >> 10) & 0x3FFFC0u) : ((wj << 6) & 0x3FFFC0u);
-                v[8 * half + j] = e2m1_sr_value(v[8 * half + j], r6);
-            }
-        }
-    }
-    uint32_t b[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b[i] = e2m1x2_rn(v[2 * i], v[2 * i + 1]);
     uint2 out;
-    out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    if constexpr (SR) {
+        const uint64_t g = n0 >> 4;
+        const Philox4 r = philox4x32_10(uint32_t(g), uint32_t(g >> 32), offset, 0u, keys);
+        const uint32_t q0 = e2m1x4_sr(v[0], v[1], v[2], v[3], r.w[0]);
+        const uint32_t q1 = e2m1x4_sr(v[4], v[5], v[6], v[7], r.w[1]);
+        const uint32_t q2 = e2m1x4_sr(v[8], v[9], v[10], v[11], r.w[2]);
+        const uint32_t q3 = e2m1x4_sr(v[12], v[13], v[14], v[15], r.w[3]);
+        out.x = q0 | (q1 << 16);
+        out.y = q2 | (q3 << 16);
+    } else {
+        uint32_t b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) b[i] = e2m1x2_rn(v[2 * i], v[2 * i + 1]);
+        out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+        out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    }
     return out;
 }
 
@@ -405,8 +404,6 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
             }
             w[m] = __byte_perm(o[0], o[1], 0x6420) | (__byte_perm(o[0], o[1], 0x7531) << 4);
         }
-        *reinterpret_cast<uint4*>(a.state + widx) = make_uint4(s[0], s[1], s[2], s[3]);
-        *reinterpret_cast<uint4*>(a.state + widx + 16) = make_uint4(s[4], s[5], s[6], s[7]);
     }
     *reinterpret_cast<uint4*>(a.codes + (widx >> 1)) = make_uint4(w[0], w[1], w[2], w[3]);
     const int64_t S = nbc;  // scales per row
@@ -426,7 +423,7 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
 constexpr int kQ2dWarps = 8;   // warps (blocks) per CTA
 
 template <typename InT, bool RHT, bool SR, bool DEOSC>
-__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kQ2dWarps * 32, 4) quant2d_kernel(QuantArgs a) {
     // Per warp: the block as 32 rows x 8 chunks of 4 binary32 (chunk c of row
     // r at slot c ^ (r & 7)), and its 32 x 32 state bytes (word c of row r at
     // slot c ^ ((r >> 2) & 7)); both swizzles keep the row-of-4-rows writes
@@ -480,6 +477,18 @@ __global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_kernel(QuantArgs a) {
         for (int j = 0; j < 8; ++j) s[j] = ss[warp][lane * 8 + (j ^ ((lane >> 2) & 7))];
     }
     quant2d_block<InT, RHT, SR, DEOSC>(a, g, bi, bj, lane, x0, x1, s);
+    if constexpr (DEOSC) {
+        // the updated state goes back through the same swizzled tile and out
+        // in the coalesced layout (rows 4k..4k+3 per instruction)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss[warp][lane * 8 + (j ^ ((lane >> 2) & 7))] = s[j];
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int rr = 4 * k + q;
+            *reinterpret_cast<uint32_t*>(a.state + (g * R + bi * 32 + rr) * C + c0 + 4 * c) = ss[warp][rr * 8 + (c ^ k)];
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -21,17 +21,41 @@ def test_philox_matches_curand(curand_philox):
     assert np.array_equal(ref, ours)
 
 
+def _rev16(u):
+    return int(format(u, "016b")[::-1], 2)
+
+
 def test_sr_bits_are_curand_words(curand_philox):
-    """Element n draws 16 bits of Philox(key=seed, ctr=(n>>3 lo, hi, offset, 0))."""
+    """Element n draws 16 bits of word (n>>2)&3 of Philox(key=seed,
+    ctr=(n>>4 lo, hi, offset, 0)): with bytes b0..b3 of that word, elements
+    4m..4m+3 take b2:b0, its bit reversal, b3:b1, its bit reversal."""
     seed, offset = 0x1234_5678_9ABC_DEF0, 7
-    ns = [0, 1, 2, 3, 7, 8, 15, 1 << 33, (1 << 40) + 5]
-    ctr = np.array([[(n >> 3) & 0xFFFFFFFF, (n >> 3) >> 32, offset, 0] for n in ns], dtype=np.uint64)
+    ns = [0, 1, 2, 3, 4, 5, 6, 7, 12, 13, 14, 15, 16, 31, 1 << 33, (1 << 40) + 5, (1 << 40) + 10]
+    ctr = np.array([[(n >> 4) & 0xFFFFFFFF, (n >> 4) >> 32, offset, 0] for n in ns], dtype=np.uint64)
     key = np.array([[seed & 0xFFFFFFFF, seed >> 32]] * len(ns), dtype=np.uint64)
     words = curand_philox(ctr, key)
     for n, w in zip(ns, words):
-        j = n & 7
-        want = (int(w[j >> 1]) >> (16 * (j & 1))) & 0xFFFF
-        assert oracle.sr_bits16(seed, offset, n) == want
+        word = int(w[(n >> 2) & 3])
+        b = [(word >> (8 * i)) & 0xFF for i in range(4)]
+        even, odd = (b[2] << 8) | b[0], (b[3] << 8) | b[1]
+        want = [even, _rev16(even), odd, _rev16(odd)][n & 3]
+        assert oracle.sr_bits16(seed, offset, n) == want, n
+
+
+def test_sr_bits_uniform_and_pairwise_uncorrelated():
+    """Every element's 16-bit draw is uniform (each bit is set half the time)
+    and the bit-reversed partner is uncorrelated with it in value."""
+    seed, offset = 5, 3
+    n = np.arange(0, 4 * 20000)
+    r = np.array([oracle.sr_bits16(seed, offset, int(i)) for i in n], dtype=np.float64)
+    for j in range(4):
+        rj = r[j::4]
+        assert abs(rj.mean() / 65536 - 0.5) < 0.01
+        for bit in (0, 7, 15):
+            assert abs(np.mean((rj.astype(np.int64) >> bit) & 1) - 0.5) < 0.02
+    for a, b in ((0, 1), (2, 3), (0, 2)):
+        c = np.corrcoef(r[a::4], r[b::4])[0, 1]
+        assert abs(c) < 0.03, (a, b, c)
 
 
 def test_rht_signs_are_curand_bits(curand_philox):
@@ -118,7 +142,8 @@ def test_rht_butterfly_order_independent_check():
 
 def test_sr_exhaustive_over_r16():
     """For fixed v the number of r16 in [0, 2^16) that round up is
-    ceil(f * 2^16): exactly the draws with r16 * 2^-16 < f."""
+    floor(f * 2^16): the draws whose sum with the kept 16-bit position
+    carries out of 16 bits.  f is computed here in binary64 from the grid."""
     grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
     rng = np.random.default_rng(12)
     for i in range(7):
@@ -127,7 +152,12 @@ def test_sr_exhaustive_over_r16():
             v = np.float32(lo + frac * (hi - lo))
             f = (float(v) - lo) / (hi - lo)
             ups = sum(1 for r in range(0, 65536) if (oracle.e2m1_sr(float(v), r) & 7) == i + 1)
-            assert ups == int(np.ceil(f * 65536))
+            assert ups == int(np.floor(f * 65536))
+            # and they are the top F draws
+            F = int(np.floor(f * 65536))
+            if 0 < F < 65536:
+                assert (oracle.e2m1_sr(float(v), 65536 - F) & 7) == i + 1
+                assert (oracle.e2m1_sr(float(v), 65535 - F) & 7) == i
 
 
 def test_sr_unbiased_over_1e6_draws():
