@@ -400,7 +400,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--experts", type=int, default=32,
                     help="smaller layers are for profiler captures only; the result line names the size")
@@ -488,28 +488,61 @@ def main():
             components[k] = {"ms": round(t, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
 
     # ---------------- end to end through the C ABI with host buffers
-    h2d_bytes = sum(t.numel() * t.element_size() for t in (layer.x, layer.h, layer.dy_up, layer.dy_down))
-    host_in = [t.cpu().pin_memory() for t in (layer.x, layer.h, layer.dy_up, layer.dy_down)]
-    host_out = [torch.empty(layer.dx.shape, dtype=torch.float32).pin_memory(),
-                torch.empty(layer.dh.shape, dtype=torch.float32).pin_memory()]
-    d2h_bytes = sum(t.numel() * t.element_size() for t in host_out)
-    dev_in = (layer.x, layer.h, layer.dy_up, layer.dy_down)
-    layer.step()
+    # Every step uploads its inputs from pinned host memory and reads its
+    # results back.  Two sets of device I/O buffers and three streams let the
+    # upload of step i+1, the step-i kernels and the download of step i-1 run
+    # at once (PCIe moves both directions concurrently).
+    io_in, io_out = ("x", "h", "dy_up", "dy_down"), ("dx", "dh")
+    sets = [{n: getattr(layer, n) for n in io_in + io_out},
+            {n: torch.empty_like(getattr(layer, n)) for n in io_in + io_out}]
+    for n in io_in:
+        sets[1][n].copy_(getattr(layer, n))
+    h2d_bytes = sum(sets[0][n].numel() * sets[0][n].element_size() for n in io_in)
+    host_in = {n: sets[0][n].cpu().pin_memory() for n in io_in}
+    host_out = {n: torch.empty(sets[0][n].shape, dtype=torch.float32).pin_memory() for n in io_out}
+    d2h_bytes = sum(t.numel() * t.element_size() for t in host_out.values())
+    s_up, s_dn = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    up_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    dn_done = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def e2e_pipeline(nsteps, e_start=None, e_end=None):
+        if e_start is not None:
+            e_start.record(s_up)
+        for i in range(nsteps):
+            b = i % 2
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(comp_done[b])          # step i-2 no longer reads buffer set b
+                for n in io_in:
+                    sets[b][n].copy_(host_in[n], non_blocking=True)
+                up_done[b].record(s_up)
+            stream.wait_event(up_done[b])
+            if i >= 2:
+                stream.wait_event(dn_done[b])              # results of step i-2 are on the host
+            for n in io_in + io_out:
+                setattr(layer, n, sets[b][n])
+            layer.step()
+            comp_done[b].record(stream)
+            with torch.cuda.stream(s_dn):
+                s_dn.wait_event(comp_done[b])
+                for n in io_out:
+                    host_out[n].copy_(sets[b][n], non_blocking=True)
+                dn_done[b].record(s_dn)
+        if e_end is not None:
+            e_end.record(s_dn)
+
+    e2e_pipeline(2)                                          # untimed pass through the pipeline
     torch.cuda.synchronize()
     barrier(pg)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        for d, h in zip(dev_in, host_in):
-            d.copy_(h, non_blocking=True)
-        layer.step()
-        host_out[0].copy_(layer.dx, non_blocking=True)
-        host_out[1].copy_(layer.dh, non_blocking=True)
-    e1.record(stream)
+    e2e_pipeline(args.e2e_steps, e0, e1)
     torch.cuda.synchronize()
     barrier(pg)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), pg, dev)
     e2e_value = step_flops * args.e2e_steps * world / (e2e_ms / 1e3) / 1e12
+    for n in io_in + io_out:
+        setattr(layer, n, sets[0][n])
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
