@@ -221,6 +221,21 @@ class Layer:
         self.step_idx += 1
 
 
+# DRAM bytes per launch on the full workload (32 experts, 16384 tokens):
+# ncu dram__bytes_read.sum + dram__bytes_write.sum of each launch of the
+# 8-expert / 4096-token layer, whose every tensor is exactly a quarter of the
+# full one, times 4.  An entry must go back to None when its kernel changes.
+DRAM_BYTES_FULL = {
+    "deosc_up": 4 * (664.1e6 + 244.8e6), "deosc_down": 4 * (332.1e6 + 107.2e6),
+    "quant_x": 4 * (97.4e6 + 8.9e6), "quant_h": 4 * (97.4e6 + 9.9e6),
+    "quant_dy_up": 4 * (194.8e6 + 36.8e6), "quant_dy_down": 4 * (97.4e6 + 9.0e6),
+    "quant_xt": 4 * (97.4e6 + 7.1e6), "quant_dy_up_t": 4 * (194.8e6 + 33.2e6),
+    "quant_ht": 4 * (97.4e6 + 4.5e6), "quant_dy_down_t": 4 * (97.4e6 + 6.6e6),
+    "fprop_up": 4 * (97.5e6 + 336.1e6), "fprop_down": 4 * (61.3e6 + 141.0e6),
+    "dgrad_up": 4 * (122.5e6 + 153.2e6), "dgrad_down": 4 * (61.3e6 + 139.5e6),
+    "wgrad_up": 4 * (78.8e6 + 472.2e6), "wgrad_down": 4 * (51.9e6 + 205.9e6),
+}
+
 KERNELS = ["deosc_up", "deosc_down", "quant_x", "fprop_up", "quant_h", "fprop_down", "quant_dy_up", "dgrad_up",
            "quant_dy_down", "dgrad_down", "quant_xt", "quant_dy_up_t", "wgrad_up", "quant_ht", "quant_dy_down_t",
            "wgrad_down"]
@@ -462,19 +477,21 @@ def main():
     fp4_peak = peaks["bf16_sustained"] * NOMINAL_FP4_OVER_BF16
     dominant = max(per_kernel, key=lambda k: per_kernel[k])
     dom_ms = per_kernel[dominant]
+    full_size = (args.experts, args.tokens) == (32, 16384)
+    dom_traffic = DRAM_BYTES_FULL.get(dominant) if full_size else None
     if dominant in layer.gemm_flops:
         achieved = layer.gemm_flops[dominant] / (dom_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak,
                 "peak_source": "%s sustained bf16 x %.0f (nominal FP4:BF16 dense ratio)" % (peaks["source"],
                                                                                           NOMINAL_FP4_OVER_BF16),
-                "kernel": dominant, "traffic": None,
+                "kernel": dominant, "traffic": dom_traffic,
                 "hbm_frac": layer.gemm_out_bytes(dominant) / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
     else:
         achieved = layer.quant_bytes[dominant] / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                "kernel": dominant, "traffic": None}
+                "kernel": dominant, "traffic": dom_traffic}
     components = {}
     for k in KERNELS:
         t = per_kernel[k]
