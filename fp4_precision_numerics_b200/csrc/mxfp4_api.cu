@@ -126,26 +126,26 @@ bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void
 
 template <typename InT>
 mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
-    // input [groups][rows = T][cols = F] with row stride ld: box = 64 features x 128 tokens
+    // input [groups][rows = T][cols = F] with row stride ld: box = 128 features x (128 or 64) tokens
     CUtensorMap tm;
     const uint64_t esz = sizeof(InT);
     const uint64_t dims[3] = {uint64_t(qa.cols), uint64_t(qa.rows), uint64_t(qa.groups)};
     const uint64_t strides[2] = {uint64_t(qa.ld) * esz, uint64_t(qa.ld) * esz * uint64_t(qa.rows)};
-    const uint32_t box[3] = {uint32_t(mxfp4::kTF), uint32_t(mxfp4::kTT), 1u};
+    const uint32_t box[3] = {uint32_t(mxfp4::kColsTF), uint32_t(mxfp4::cols_tt<InT>()), 1u};
     if (!make_map_plain(&tm, sizeof(InT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
                         qa.in, dims, strides, box))
         return fail(MXFP4_ERR_CUDA, "mxfp4_quantize(along rows): tensor map encode failed");
     uint32_t* status = status_word();
     if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_quantize: cannot resolve the device status word");
-    const int64_t tiles = qa.groups * ((qa.rows + mxfp4::kTT - 1) / mxfp4::kTT) *
-                          ((qa.cols + mxfp4::kTF - 1) / mxfp4::kTF);
+    const int64_t tt = mxfp4::cols_tt<InT>(), tf = mxfp4::kColsTF;
+    const int64_t tiles = qa.groups * ((qa.rows + tt - 1) / tt) * ((qa.cols + tf - 1) / tf);
     const int64_t cap = int64_t(num_sms()) * 4;
     const unsigned grid = unsigned(tiles < cap ? tiles : cap);
     const uint32_t smem = mxfp4::cols_smem_bytes<InT>();
     auto go = [&](auto kern) -> mxfp4_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return fail(MXFP4_ERR_CUDA, "mxfp4_quantize(along rows): shared-memory attribute");
-        kern<<<grid, 256, smem, st>>>(tm, qa, status);
+        kern<<<grid, mxfp4::cols_threads<InT>(), smem, st>>>(tm, qa, status);
         return check_launch("mxfp4_quantize(1d along rows)");
     };
     if (rht && sr) return go(mxfp4::quant1d_cols_kernel<InT, true, true>);

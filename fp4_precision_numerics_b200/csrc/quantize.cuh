@@ -101,6 +101,29 @@ __device__ __forceinline__ void rht16(float (&x)[16], uint32_t signs) {
     }
 }
 
+// rht16 on two independent 16-element chunks at once, held as packed pairs
+// (chunk A in the low halves, chunk B in the high halves): every operation
+// is the scalar one of rht16 applied to both halves.
+__device__ __forceinline__ void rht16x2(uint64_t (&p)[16], uint32_t signs) {
+    const uint64_t quarter = f2_pack(0.25f, 0.25f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t sbit = uint64_t((signs >> i) & 1u) << 31;
+        p[i] = f2_mul(p[i] ^ (sbit | (sbit << 32)), quarter);
+    }
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if ((i & h) == 0) {
+                const uint64_t a = p[i], b = p[i + h];
+                p[i] = f2_add(a, b);
+                p[i + h] = f2_sub(a, b);
+            }
+        }
+    }
+}
+
 __device__ __forceinline__ float amax16(const float (&x)[16]) {
     float m = 0.0f;
 #pragma unroll
@@ -113,11 +136,8 @@ __device__ __forceinline__ float amax16(const float (&x)[16]) {
 // covers the 16 elements, word j the four elements 4j..4j+3, consumed by the
 // four-element stochastic-rounding conversion (see e2m1x4_sr).
 template <bool SR>
-__device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, const PhiloxKeys& keys,
-                                         uint32_t offset) {
-    float v[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(x[i], inv_scale);
+__device__ __forceinline__ uint2 quant16_scaled(const float (&v)[16], uint64_t n0, const PhiloxKeys& keys,
+                                                uint32_t offset) {
     uint2 out;
     if constexpr (SR) {
         const uint64_t g = n0 >> 4;
@@ -136,6 +156,15 @@ __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, 
         out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
     }
     return out;
+}
+
+template <bool SR>
+__device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, const PhiloxKeys& keys,
+                                         uint32_t offset) {
+    float v[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(x[i], inv_scale);
+    return quant16_scaled<SR>(v, n0, keys, offset);
 }
 
 // ---------------------------------------------------------------------------
@@ -182,25 +211,36 @@ __global__ void __launch_bounds__(256) quant1d_rows_kernel(QuantArgs a) {
 
 // ---------------------------------------------------------------------------
 // 1D blocks along dim 0 (the token dim), output transposed: input [T, F]
-// (per group), output [F, T].  Persistent CTAs walk 128-token x 64-feature
-// tiles; a 3-deep ring of shared-memory buffers is filled by TMA (zero fill
-// at the ragged edges), so the next tiles stream in while the current one
-// is quantised.  Each thread owns one (feature, 32-token block): RHT on its
-// two 16-token chunks, amax, scale, rounding, one 16-byte store of codes.
+// (per group), output [F, T].  Persistent CTAs walk tiles of 128 features x
+// (128 tokens for bf16, 64 for binary32), 32 KB each; a 3-deep ring of
+// shared-memory buffers is filled by TMA (zero fill at the ragged edges), so
+// the next tiles stream in while the current one is quantised.  Each thread
+// owns two neighbouring features of one 32-token block: one 4-byte (bf16) or
+// 8-byte (binary32) shared load per token gives both, and the RHT and the
+// scaling run on packed pairs (two-wide fp32); then per feature the amax,
+// scale, rounding and a 16-byte store of codes.
 // ---------------------------------------------------------------------------
-constexpr int kTT = 128;    // tokens per tile
-constexpr int kTF = 64;     // features per tile
+constexpr int kColsTF = 128;   // features per tile
 constexpr int kColsRing = 3;
 
 template <typename InT>
-__host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(kTT * kTF * sizeof(InT)); }
+__host__ __device__ constexpr int cols_tt() { return sizeof(InT) == 2 ? 128 : 64; }   // tokens per tile
+
+template <typename InT>
+__host__ __device__ constexpr int cols_threads() { return (kColsTF / 2) * (cols_tt<InT>() / 32); }
+
+template <typename InT>
+__host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(cols_tt<InT>() * kColsTF * sizeof(InT)); }
 
 template <typename InT>
 __host__ __device__ constexpr uint32_t cols_smem_bytes() { return kColsRing * cols_tile_bytes<InT>() + 64 + 128; }
 
 template <typename InT, bool RHT, bool SR>
-__global__ void __launch_bounds__(256) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
+__global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
                                                            uint32_t* status) {
+    constexpr int kTT = cols_tt<InT>();
+    constexpr int kTF = kColsTF;
+    constexpr int kPairs = kTF / 2;
     extern __shared__ uint8_t cols_smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(cols_smem_raw) + 127) & ~uintptr_t(127));
     constexpr uint32_t kTile = cols_tile_bytes<InT>();
@@ -233,8 +273,8 @@ __global__ void __launch_bounds__(256) quant1d_cols_kernel(const __grid_constant
     __syncthreads();
     PhiloxKeys keys;
     if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
-    const int fl = threadIdx.x & 63;
-    const int blk = threadIdx.x >> 6;
+    const int pr = threadIdx.x % kPairs;   // features 2 pr, 2 pr + 1 of the tile
+    const int blk = threadIdx.x / kPairs;  // 32-token block of the tile
     const int64_t S = T >> 5;
     for (int64_t i = 0; i < mine; ++i) {
         const int b = int(i % kColsRing);
@@ -242,35 +282,56 @@ __global__ void __launch_bounds__(256) quant1d_cols_kernel(const __grid_constant
         const bool got = mbar_wait_bounded(&full[b], phase, abort_flag, status, kRoleProducer);
         int64_t g, t0, f0;
         tile_coords(i, g, t0, f0);
-        const int64_t f = f0 + fl;
+        const int64_t f = f0 + 2 * pr;
         const int64_t tb = t0 + blk * 32;
         if (got && f < F && tb < T) {
-            const InT* tile = reinterpret_cast<const InT*>(smem + b * kTile);   // [kTT][kTF], dense
-            float x0[16], x1[16];
+            const uint8_t* tile = smem + b * kTile;   // [kTT][kTF] of InT, dense
+            uint64_t p[32];                            // token k: (feature f, feature f + 1)
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
+            for (int k = 0; k < 32; ++k) {
+                const int e = (blk * 32 + k) * kTF + 2 * pr;
                 if constexpr (sizeof(InT) == 2) {
-                    x0[k] = __uint_as_float(uint32_t(tile[(blk * 32 + k) * kTF + fl]) << 16);
-                    x1[k] = __uint_as_float(uint32_t(tile[(blk * 32 + 16 + k) * kTF + fl]) << 16);
+                    const uint32_t w = *reinterpret_cast<const uint32_t*>(tile + 2 * e);
+                    p[k] = f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
                 } else {
-                    x0[k] = tile[(blk * 32 + k) * kTF + fl];
-                    x1[k] = tile[(blk * 32 + 16 + k) * kTF + fl];
+                    p[k] = *reinterpret_cast<const uint64_t*>(tile + 4 * e);
                 }
             }
             if constexpr (RHT) {
-                rht16(x0, a.rht_signs);
-                rht16(x1, a.rht_signs);
+                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[0]), a.rht_signs);
+                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[16]), a.rht_signs);
             }
-            const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
-            const float inv = inv_scale_from_byte(sb);
-            const int64_t orow = g * F + f;  // output row (groups back to back)
-            const uint64_t n0 = uint64_t(orow) * uint64_t(T) + uint64_t(tb);
-            const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
-            const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
-            *reinterpret_cast<uint4*>(a.codes + orow * (T >> 1) + (tb >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+            float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+                float lo, hi;
+                f2_unpack(p[k], lo, hi);
+                m0 = fmaxf(m0, fabsf(lo));
+                m1 = fmaxf(m1, fabsf(hi));
+            }
+            const int sb0 = scale_byte_from_amax(m0), sb1 = scale_byte_from_amax(m1);
+            const uint64_t inv = f2_pack(inv_scale_from_byte(sb0), inv_scale_from_byte(sb1));
+            float v0[32], v1[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) f2_unpack(f2_mul(p[k], inv), v0[k], v1[k]);
+            const bool two = f + 1 < F;
+            const int64_t orow = g * F + f;  // output row of feature f (groups back to back)
             const int64_t s = tb >> 5;
-            if (a.scales) a.scales[orow * S + s] = uint8_t(sb);
-            if (a.scales_mma) a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f, s, S)] = uint8_t(sb);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !two) break;
+                const float* v = h ? v1 : v0;
+                const uint64_t n0 = uint64_t(orow + h) * uint64_t(T) + uint64_t(tb);
+                const uint2 q0 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v), n0, keys, a.sr_offset);
+                const uint2 q1 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v + 16), n0 + 16, keys,
+                                                    a.sr_offset);
+                *reinterpret_cast<uint4*>(a.codes + (orow + h) * (T >> 1) + (tb >> 1)) =
+                    make_uint4(q0.x, q0.y, q1.x, q1.y);
+                const int sb = h ? sb1 : sb0;
+                if (a.scales) a.scales[(orow + h) * S + s] = uint8_t(sb);
+                if (a.scales_mma)
+                    a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f + h, s, S)] = uint8_t(sb);
+            }
         }
         __syncthreads();  // buffer b fully read: refill it with tile i + kColsRing
         if (threadIdx.x == 0 && i + kColsRing < mine) {
