@@ -119,7 +119,7 @@ class Layer:
         self.dw_up = torch.empty((E, F, D), **f32)
         self.dw_down = torch.empty((E, D, D), **f32)
         self.step_idx = 0
-        self.launches_per_step = 16
+        self.launches_per_step = 12
         # algorithmic work
         r = self.rows_real
         self.gemm_flops = {
@@ -127,13 +127,13 @@ class Layer:
             "dgrad_up": 2.0 * r * F * D, "dgrad_down": 2.0 * r * D * D,
             "wgrad_up": 2.0 * r * F * D, "wgrad_down": 2.0 * r * D * D,
         }
-        # quantise bytes: read input, write codes (1/2 B) + scales (1/32 B); de-osc adds state r/w
-        q1 = 2.0 + 0.5 + 1.0 / 32
+        # quantise bytes: the dual quantiser reads its bf16 input once and writes
+        # codes (1/2 B) + scales (1/32 B) in each direction; de-osc adds state r/w
+        q2 = 2.0 + 2 * (0.5 + 1.0 / 32)
         self.quant_bytes = {
             "deosc_up": E * F * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
             "deosc_down": E * D * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
-            "quant_x": M * D * q1, "quant_h": M * D * q1, "quant_dy_up": M * F * q1, "quant_dy_down": M * D * q1,
-            "quant_xt": M * D * q1, "quant_ht": M * D * q1, "quant_dy_up_t": M * F * q1, "quant_dy_down_t": M * D * q1,
+            "dual_x": M * D * q2, "dual_h": M * D * q2, "dual_dy_up": M * F * q2, "dual_dy_down": M * D * q2,
         }
         self.gemm_dims = {
             "fprop_up": (M, F, D), "fprop_down": (M, D, D), "dgrad_up": (M, D, F), "dgrad_down": (M, D, D),
@@ -168,52 +168,43 @@ class Layer:
                         out=q["w_down"])
         rec("deosc_down", 1)
         M = self.M
-        rec("quant_x", 0)
-        mx.quantize(self.x, scales=False, scales_mma=True, out=q["x"])
-        rec("quant_x", 1)
+        # activations and gradients: one dual-direction quantisation each gives
+        # the contraction-dim operand (fprop/dgrad) and the token-dim RHT operand (wgrad)
+        rec("dual_x", 0)
+        mx.quantize_dual(self.x, col_rht_seed=1, scales=False, scales_mma=True, out_row=q["x"], out_col=q["xt"])
+        rec("dual_x", 1)
         rec("fprop_up", 0)
         mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["x"]["codes"], q["x"]["scales_mma"], q["w_up"]["codes"],
                         q["w_up"]["scales_mma"], M, F, D, out=self.y_up)
         rec("fprop_up", 1)
-        rec("quant_h", 0)
-        mx.quantize(self.h, scales=False, scales_mma=True, out=q["h"])
-        rec("quant_h", 1)
+        rec("dual_h", 0)
+        mx.quantize_dual(self.h, col_rht_seed=1, scales=False, scales_mma=True, out_row=q["h"], out_col=q["ht"])
+        rec("dual_h", 1)
         rec("fprop_down", 0)
         mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["h"]["codes"], q["h"]["scales_mma"], q["w_down"]["codes"],
                         q["w_down"]["scales_mma"], M, D, D, out=self.y_down)
         rec("fprop_down", 1)
-        rec("quant_dy_up", 0)
-        mx.quantize(self.dy_up, sr_seed=1, sr_offset=2 * s, scales=False, scales_mma=True, out=q["dy_up"])
-        rec("quant_dy_up", 1)
+        rec("dual_dy_up", 0)
+        mx.quantize_dual(self.dy_up, col_rht_seed=1, sr_seed=1, row_sr_offset=2 * s, col_sr_offset=1000 + 2 * s,
+                         scales=False, scales_mma=True, out_row=q["dy_up"], out_col=q["dy_up_t"])
+        rec("dual_dy_up", 1)
         rec("dgrad_up", 0)
         mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_up"]["codes"], q["dy_up"]["scales_mma"],
                         q["w_up"]["codes_t"], q["w_up"]["scales_mma_t"], M, D, F, out=self.dx)
         rec("dgrad_up", 1)
-        rec("quant_dy_down", 0)
-        mx.quantize(self.dy_down, sr_seed=1, sr_offset=2 * s + 1, scales=False, scales_mma=True, out=q["dy_down"])
-        rec("quant_dy_down", 1)
+        rec("dual_dy_down", 0)
+        mx.quantize_dual(self.dy_down, col_rht_seed=1, sr_seed=1, row_sr_offset=2 * s + 1,
+                         col_sr_offset=1001 + 2 * s, scales=False, scales_mma=True, out_row=q["dy_down"],
+                         out_col=q["dy_down_t"])
+        rec("dual_dy_down", 1)
         rec("dgrad_down", 0)
         mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_down"]["codes"], q["dy_down"]["scales_mma"],
                         q["w_down"]["codes_t"], q["w_down"]["scales_mma_t"], M, D, D, out=self.dh)
         rec("dgrad_down", 1)
-        rec("quant_xt", 0)
-        mx.quantize(self.x, along_rows=True, rht_seed=1, scales=False, scales_mma=True, out=q["xt"])
-        rec("quant_xt", 1)
-        rec("quant_dy_up_t", 0)
-        mx.quantize(self.dy_up, along_rows=True, rht_seed=1, sr_seed=1, sr_offset=1000 + 2 * s, scales=False,
-                    scales_mma=True, out=q["dy_up_t"])
-        rec("quant_dy_up_t", 1)
         rec("wgrad_up", 0)
         mx.grouped_gemm(mx.GEMM_WGRAD, self.offsets, q["dy_up_t"]["codes"], q["dy_up_t"]["scales_mma"],
                         q["xt"]["codes"], q["xt"]["scales_mma"], F, D, M, out=self.dw_up)
         rec("wgrad_up", 1)
-        rec("quant_ht", 0)
-        mx.quantize(self.h, along_rows=True, rht_seed=1, scales=False, scales_mma=True, out=q["ht"])
-        rec("quant_ht", 1)
-        rec("quant_dy_down_t", 0)
-        mx.quantize(self.dy_down, along_rows=True, rht_seed=1, sr_seed=1, sr_offset=1001 + 2 * s, scales=False,
-                    scales_mma=True, out=q["dy_down_t"])
-        rec("quant_dy_down_t", 1)
         rec("wgrad_down", 0)
         mx.grouped_gemm(mx.GEMM_WGRAD, self.offsets, q["dy_down_t"]["codes"], q["dy_down_t"]["scales_mma"],
                         q["ht"]["codes"], q["ht"]["scales_mma"], D, D, M, out=self.dw_down)
@@ -227,35 +218,49 @@ class Layer:
 # full one, times 4.  An entry must go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
     "deosc_up": 4 * (664.1e6 + 244.8e6), "deosc_down": 4 * (332.1e6 + 107.2e6),
-    "quant_x": 4 * (97.4e6 + 8.9e6), "quant_h": 4 * (97.4e6 + 9.9e6),
-    "quant_dy_up": 4 * (194.8e6 + 36.8e6), "quant_dy_down": 4 * (97.4e6 + 9.0e6),
-    "quant_xt": 4 * (97.4e6 + 7.1e6), "quant_dy_up_t": 4 * (194.8e6 + 33.2e6),
-    "quant_ht": 4 * (97.4e6 + 4.5e6), "quant_dy_down_t": 4 * (97.4e6 + 6.6e6),
+    "dual_x": None, "dual_h": None, "dual_dy_up": None, "dual_dy_down": None,
     "fprop_up": 4 * (97.5e6 + 336.1e6), "fprop_down": 4 * (61.3e6 + 141.0e6),
     "dgrad_up": 4 * (122.5e6 + 153.2e6), "dgrad_down": 4 * (61.3e6 + 139.5e6),
     "wgrad_up": 4 * (78.8e6 + 472.2e6), "wgrad_down": 4 * (51.9e6 + 205.9e6),
 }
 
-KERNELS = ["deosc_up", "deosc_down", "quant_x", "fprop_up", "quant_h", "fprop_down", "quant_dy_up", "dgrad_up",
-           "quant_dy_down", "dgrad_down", "quant_xt", "quant_dy_up_t", "wgrad_up", "quant_ht", "quant_dy_down_t",
-           "wgrad_down"]
+KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
+           "dual_dy_down", "dgrad_down", "wgrad_up", "wgrad_down"]
 
 
 # ---------------------------------------------------------------------------
 # Clock sampling
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of one GPU, sampled during
+    the timed region: through NVML every ~5 ms, else `nvidia-smi -lms 50`.
+    It only reads; no setting of the GPU is touched."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
-        self.samples = []
+        self.samples = []          # (time, sm_mhz, max_mhz, set of reasons)
         self.proc = None
         self.thread = None
+        self.stop_flag = threading.Event()
 
     def start(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(self.gpu_id)
+            h = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid.startswith("GPU-")
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(uuid)))
+            self.thread = threading.Thread(target=self._nvml, args=(pynvml, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + self.FIELDS,
                                           "--format=csv,noheader,nounits", "-lms", "50"], stdout=subprocess.PIPE,
@@ -266,11 +271,35 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _nvml(self, pynvml, h):
+        get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop_flag.is_set():
+            try:
+                mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                bits = get_reasons(h)
+            except Exception:
+                break
+            reasons = {n for n, b in self.REASON_BITS.items() if bits & b}
+            self.samples.append((time.time(), float(mhz), float(max_mhz), reasons))
+            time.sleep(0.005)
+
     def _read(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                mhz, maxmhz = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(names, parts[4:8]) if v.lower().startswith("active")}
+            self.samples.append((time.time(), mhz, maxmhz, reasons))
 
     def stop(self):
+        self.stop_flag.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -281,25 +310,14 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self, t0, t1):
-        rows = [s for (t, s) in self.samples if t0 - 0.05 <= t <= t1 + 0.05] or [s for (_, s) in self.samples]
-        mhz, maxmhz, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            parts = [p.strip() for p in r.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                mhz.append(float(parts[0]))
-                maxmhz.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not mhz:
+        rows = [r for r in self.samples if t0 <= r[0] <= t1] or self.samples
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxmhz), "reasons": sorted(reasons),
-                "samples": len(mhz)}
+        reasons = set()
+        for r in rows:
+            reasons |= r[3]
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
 
 
 # ---------------------------------------------------------------------------
@@ -412,7 +430,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=8)

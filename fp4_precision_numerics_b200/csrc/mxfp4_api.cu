@@ -154,6 +154,42 @@ mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
     return go(mxfp4::quant1d_cols_kernel<InT, false, false>);
 }
 
+template <typename InT>
+mxfp4_status launch_dual(const mxfp4::QuantArgs& qa, bool rht_col, bool rht_row, bool sr, cudaStream_t st) {
+    CUtensorMap tm;
+    const uint64_t esz = sizeof(InT);
+    const uint64_t dims[3] = {uint64_t(qa.cols), uint64_t(qa.rows), uint64_t(qa.groups)};
+    const uint64_t strides[2] = {uint64_t(qa.ld) * esz, uint64_t(qa.ld) * esz * uint64_t(qa.rows)};
+    const uint32_t box[3] = {uint32_t(mxfp4::kColsTF), uint32_t(mxfp4::cols_tt<InT>()), 1u};
+    if (!make_map_plain(&tm, sizeof(InT) == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                        qa.in, dims, strides, box))
+        return fail(MXFP4_ERR_CUDA, "mxfp4_quantize_dual: tensor map encode failed");
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_quantize_dual: cannot resolve the device status word");
+    const int64_t tt = mxfp4::cols_tt<InT>(), tf = mxfp4::kColsTF;
+    const int64_t tiles = qa.groups * ((qa.rows + tt - 1) / tt) * ((qa.cols + tf - 1) / tf);
+    const int64_t cap = int64_t(num_sms()) * 4;
+    const unsigned grid = unsigned(tiles < cap ? tiles : cap);
+    const uint32_t smem = mxfp4::cols_smem_bytes<InT>();
+    auto go = [&](auto kern) -> mxfp4_status {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+            return fail(MXFP4_ERR_CUDA, "mxfp4_quantize_dual: shared-memory attribute");
+        kern<<<grid, mxfp4::cols_threads<InT>(), smem, st>>>(tm, qa, status);
+        return check_launch("mxfp4_quantize_dual");
+    };
+    using namespace mxfp4;
+    if (sr) {
+        if (rht_col && rht_row) return go(quant1d_cols_kernel<InT, true, true, true, true>);
+        if (rht_col) return go(quant1d_cols_kernel<InT, true, true, true, false>);
+        if (rht_row) return go(quant1d_cols_kernel<InT, false, true, true, true>);
+        return go(quant1d_cols_kernel<InT, false, true, true, false>);
+    }
+    if (rht_col && rht_row) return go(quant1d_cols_kernel<InT, true, false, true, true>);
+    if (rht_col) return go(quant1d_cols_kernel<InT, true, false, true, false>);
+    if (rht_row) return go(quant1d_cols_kernel<InT, false, false, true, true>);
+    return go(quant1d_cols_kernel<InT, false, false, true, false>);
+}
+
 template <typename InT, bool DEOSC>
 mxfp4_status launch_2d(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
     const int64_t nblocks = qa.groups * (qa.rows / 32) * (qa.cols / 32);
@@ -323,6 +359,61 @@ mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_
     if (along_rows)
         return in_dtype == MXFP4_DTYPE_BF16 ? launch_cols<uint16_t>(qa, rht, sr, st) : launch_cols<float>(qa, rht, sr, st);
     return in_dtype == MXFP4_DTYPE_BF16 ? launch_rows<uint16_t>(qa, rht, sr, st) : launch_rows<float>(qa, rht, sr, st);
+}
+
+mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, int64_t rows, int64_t cols, int64_t ld,
+                                 const mxfp4_quant_params* rp, const mxfp4_quant_params* cp,
+                                 const mxfp4_quant_outputs* row_out, const mxfp4_quant_outputs* col_out, void* stream) {
+    if (!rp || !cp) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: null params");
+    if (in_dtype != MXFP4_DTYPE_BF16 && in_dtype != MXFP4_DTYPE_F32)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: bad in_dtype %d", in_dtype);
+    if (groups < 0 || rows < 0 || cols < 0 || ld < cols)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: bad geometry");
+    if (rp->block != MXFP4_BLOCK_1X32 || cp->block != MXFP4_BLOCK_1X32)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: both directions use 1x32 blocks");
+    if (rp->along_rows != 0 || cp->along_rows != 1)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: row_params.along_rows must be 0, col_params 1");
+    if ((rp->rht_d != 0 && rp->rht_d != 16) || (cp->rht_d != 0 && cp->rht_d != 16))
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: rht_d must be 0 or 16");
+    if ((rp->rounding != MXFP4_ROUND_NEAREST && rp->rounding != MXFP4_ROUND_STOCHASTIC) ||
+        rp->rounding != cp->rounding)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: both directions need the same valid rounding");
+    const bool sr = rp->rounding == MXFP4_ROUND_STOCHASTIC;
+    if (sr && rp->sr_seed != cp->sr_seed)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: both directions need the same sr_seed");
+    const bool empty = groups == 0 || rows == 0 || cols == 0;
+    if (!in && !empty) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_quantize_dual: null input");
+    if (empty) return ok();
+    mxfp4_status s = check_outputs(row_out, false);
+    if (s != MXFP4_OK) return s;
+    s = check_outputs(col_out, false);
+    if (s != MXFP4_OK) return s;
+    if (rows % 32 || cols % 32)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize_dual: rows and cols must be multiples of 32");
+    const int esz = in_dtype == MXFP4_DTYPE_BF16 ? 2 : 4;
+    if (!aligned16(in) || (ld * esz) % 16)
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_quantize_dual: input rows not 16-byte aligned");
+    mxfp4::QuantArgs qa{};
+    qa.in = in;
+    qa.groups = groups;
+    qa.rows = rows;
+    qa.cols = cols;
+    qa.ld = ld;
+    qa.rht_signs = cp->rht_d == 16 ? rht_sign_mask(cp->rht_seed) : 0u;
+    qa.sr_key0 = uint32_t(cp->sr_seed);
+    qa.sr_key1 = uint32_t(cp->sr_seed >> 32);
+    qa.sr_offset = cp->sr_offset;
+    qa.codes = col_out->codes;
+    qa.scales = col_out->scales;
+    qa.scales_mma = col_out->scales_mma;
+    qa.r_codes = row_out->codes;
+    qa.r_scales = row_out->scales;
+    qa.r_scales_mma = row_out->scales_mma;
+    qa.r_rht_signs = rp->rht_d == 16 ? rht_sign_mask(rp->rht_seed) : 0u;
+    qa.r_sr_offset = rp->sr_offset;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return in_dtype == MXFP4_DTYPE_BF16 ? launch_dual<uint16_t>(qa, cp->rht_d == 16, rp->rht_d == 16, sr, st)
+                                        : launch_dual<float>(qa, cp->rht_d == 16, rp->rht_d == 16, sr, st);
 }
 
 mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int d, uint64_t seed,

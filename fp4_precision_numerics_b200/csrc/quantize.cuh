@@ -42,6 +42,13 @@ struct QuantArgs {
     // de-oscillation
     uint8_t* state;
     uint32_t step, flip_threshold, reset_period;
+    // dual-direction quantisation: the 1x32-along-cols outputs of the same
+    // input (codes [groups*rows, cols/2], scales, tensor-core scales)
+    uint8_t* r_codes;
+    uint8_t* r_scales;
+    uint8_t* r_scales_mma;
+    uint32_t r_rht_signs;
+    uint32_t r_sr_offset;
 };
 
 // ---------------------------------------------------------------------------
@@ -235,7 +242,11 @@ __host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(cols_
 template <typename InT>
 __host__ __device__ constexpr uint32_t cols_smem_bytes() { return kColsRing * cols_tile_bytes<InT>() + 64 + 128; }
 
-template <typename InT, bool RHT, bool SR>
+// Dual mode (DUAL): every tile is also quantised in 1x32 blocks along the
+// features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
+// the input feeds both the contraction-dim codes and the token-dim codes.
+// Each thread takes two of the tile's (token row, 32-feature block) pairs.
+template <typename InT, bool RHT, bool SR, bool DUAL = false, bool RHT_R = false>
 __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
                                                            uint32_t* status) {
     constexpr int kTT = cols_tt<InT>();
@@ -331,6 +342,69 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                 if (a.scales) a.scales[(orow + h) * S + s] = uint8_t(sb);
                 if (a.scales_mma)
                     a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f + h, s, S)] = uint8_t(sb);
+            }
+        }
+        if constexpr (DUAL) {
+            // the same tile, 1x32 blocks along the features
+            constexpr int kChunks16 = 32 * int(sizeof(InT)) / 16;   // 16-byte chunks per 32-element block
+            const int64_t SF = F >> 5;
+            const uint8_t* tile = smem + b * kTile;
+#pragma unroll 1
+            for (int e = threadIdx.x; e < kTT * (kTF / 32); e += blockDim.x) {
+                const int rr = e / (kTF / 32), fb = e % (kTF / 32);
+                const int64_t t = t0 + rr, fc = f0 + 32 * fb;
+                if (!got || t >= T || fc >= F) continue;
+                const uint8_t* src = tile + (rr * kTF + 32 * fb) * int(sizeof(InT));
+                // bf16: a block is 4 chunks of 16 bytes and half a 128-byte bank
+                // row.  Lane l of an 8-lane phase reads chunk j ^ m at step j,
+                // m = (fb >> 1) | 2 (rr & 1), so the phase covers 8 distinct
+                // 16-byte bank groups; two predicated swap stages restore the
+                // order (no register array indexed at run time).
+                uint4 w[kChunks16];
+                const int m = sizeof(InT) == 2 ? (((fb >> 1) | ((rr & 1) << 1)) & 3) : 0;
+#pragma unroll
+                for (int j = 0; j < kChunks16; ++j) w[j] = *reinterpret_cast<const uint4*>(src + 16 * (j ^ m));
+                if constexpr (sizeof(InT) == 2) {
+                    if (m & 1) {
+                        const uint4 t01 = w[0], t23 = w[2];
+                        w[0] = w[1]; w[1] = t01; w[2] = w[3]; w[3] = t23;
+                    }
+                    if (m & 2) {
+                        const uint4 t0 = w[0], t1 = w[1];
+                        w[0] = w[2]; w[1] = w[3]; w[2] = t0; w[3] = t1;
+                    }
+                }
+                float x[32];
+#pragma unroll
+                for (int j = 0; j < kChunks16; ++j) {
+                    const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+                    if constexpr (sizeof(InT) == 2) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            x[8 * j + 2 * q] = __uint_as_float(ww[q] << 16);
+                            x[8 * j + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) x[4 * j + q] = __uint_as_float(ww[q]);
+                    }
+                }
+                float (&x0)[16] = *reinterpret_cast<float(*)[16]>(&x[0]);
+                float (&x1)[16] = *reinterpret_cast<float(*)[16]>(&x[16]);
+                if constexpr (RHT_R) {
+                    rht16(x0, a.r_rht_signs);
+                    rht16(x1, a.r_rht_signs);
+                }
+                const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
+                const float inv = inv_scale_from_byte(sb);
+                const int64_t row = g * T + t;   // output row (groups back to back)
+                const uint64_t n0 = uint64_t(row) * uint64_t(F) + uint64_t(fc);
+                const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.r_sr_offset);
+                const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.r_sr_offset);
+                *reinterpret_cast<uint4*>(a.r_codes + row * (F >> 1) + (fc >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                const int64_t s = fc >> 5;
+                if (a.r_scales) a.r_scales[row * SF + s] = uint8_t(sb);
+                if (a.r_scales_mma) a.r_scales_mma[g * mma_scale_bytes(T, SF) + mma_scale_offset(t, s, SF)] = uint8_t(sb);
             }
         }
         __syncthreads();  // buffer b fully read: refill it with tile i + kColsRing

@@ -72,6 +72,10 @@ def lib() -> ctypes.CDLL:
             L.mxfp4_quantize.argtypes = [vp, st, i64, i64, i64, i64, ctypes.POINTER(QuantParams),
                                          ctypes.POINTER(QuantOutputs), vp]
             L.mxfp4_quantize.restype = st
+            L.mxfp4_quantize_dual.argtypes = [vp, st, i64, i64, i64, i64, ctypes.POINTER(QuantParams),
+                                              ctypes.POINTER(QuantParams), ctypes.POINTER(QuantOutputs),
+                                              ctypes.POINTER(QuantOutputs), vp]
+            L.mxfp4_quantize_dual.restype = st
             L.mxfp4_rht.argtypes = [vp, st, i64, i64, i64, st, ctypes.c_uint64, vp, st, vp]
             L.mxfp4_rht.restype = st
             L.mxfp4_deosc_update.argtypes = [vp, i64, i64, i64, ctypes.c_uint32, ctypes.POINTER(DeoscParams), vp,
@@ -129,6 +133,13 @@ def mxfp4_quantize(x_ptr, in_dtype, groups, rows, cols, ld, params: QuantParams,
                    stream=None):
     _check(lib().mxfp4_quantize(x_ptr, in_dtype, groups, rows, cols, ld, ctypes.byref(params),
                                 ctypes.byref(outputs), _stream(stream)))
+
+
+def mxfp4_quantize_dual(x_ptr, in_dtype, groups, rows, cols, ld, row_params: QuantParams, col_params: QuantParams,
+                        row_outputs: QuantOutputs, col_outputs: QuantOutputs, stream=None):
+    _check(lib().mxfp4_quantize_dual(x_ptr, in_dtype, groups, rows, cols, ld, ctypes.byref(row_params),
+                                     ctypes.byref(col_params), ctypes.byref(row_outputs), ctypes.byref(col_outputs),
+                                     _stream(stream)))
 
 
 def mxfp4_rht(x_ptr, in_dtype, rows, cols, ld, d, seed, out_ptr, out_dtype, stream=None):
@@ -193,6 +204,41 @@ def quantize(x: torch.Tensor, block: str = "1x32", along_rows: bool = False, rht
                         _ptr(o.get("codes_t")), _ptr(o.get("scales_mma_t")))
     mxfp4_quantize(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), G, R, C, ld, p, outs, stream)
     return o
+
+
+def quantize_dual(x: torch.Tensor, row_rht_seed=None, col_rht_seed=None, sr_seed=None, row_sr_offset: int = 0,
+                  col_sr_offset: int = 0, scales: bool = True, scales_mma: bool = False, out_row: dict | None = None,
+                  out_col: dict | None = None, stream=None) -> tuple:
+    """Quantise a [rows, cols] or [groups, rows, cols] bf16/f32 CUDA tensor
+    in both 1D directions from one read: returns (row, col), the outputs of
+    quantize(x, ...) along the last dim and quantize(x, along_rows=True, ...),
+    each a dict like quantize's."""
+    if x.dim() == 2:
+        x = x.unsqueeze(0)
+    assert x.is_cuda and x.dim() == 3 and x.stride(2) == 1
+    assert x.shape[0] == 1 or x.stride(0) == x.shape[1] * x.stride(1), "groups must be back to back"
+    G, R, C = x.shape
+    rounding = ROUND_STOCHASTIC if sr_seed is not None else ROUND_NEAREST
+    rp = QuantParams(BLOCK_1X32, 0, 16 if row_rht_seed is not None else 0, int(row_rht_seed or 0), rounding,
+                     int(sr_seed or 0), int(row_sr_offset))
+    cp = QuantParams(BLOCK_1X32, 1, 16 if col_rht_seed is not None else 0, int(col_rht_seed or 0), rounding,
+                     int(sr_seed or 0), int(col_sr_offset))
+    dev = x.device
+    outs = []
+    for (o, Ro, Co) in ((dict(out_row or {}), R, C), (dict(out_col or {}), C, R)):
+        if "codes" not in o:
+            o["codes"] = torch.empty((G, Ro, Co // 2), dtype=torch.uint8, device=dev)
+        if scales and "scales" not in o:
+            o["scales"] = torch.empty((G, Ro, Co // 32), dtype=torch.uint8, device=dev)
+        if scales_mma and "scales_mma" not in o:
+            o["scales_mma"] = torch.empty((G, mxfp4_mma_scale_bytes(Ro, Co // 32)), dtype=torch.uint8, device=dev)
+        outs.append(o)
+    ro, co = outs
+    qo_r = QuantOutputs(ro["codes"].data_ptr(), _ptr(ro.get("scales")), _ptr(ro.get("scales_mma")), None, None)
+    qo_c = QuantOutputs(co["codes"].data_ptr(), _ptr(co.get("scales")), _ptr(co.get("scales_mma")), None, None)
+    mxfp4_quantize_dual(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), G, R, C, x.stride(1), rp, cp, qo_r, qo_c,
+                        stream)
+    return ro, co
 
 
 def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, stream=None) -> torch.Tensor:

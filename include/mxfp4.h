@@ -138,6 +138,28 @@ MXFP4_API mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t grou
                             int64_t ld, const mxfp4_quant_params* params, const mxfp4_quant_outputs* out,
                             void* stream);
 
+/* Quantise one activation or gradient tensor in both 1D directions from a
+ * single read of the input: the contraction-dim codes (1x32 blocks along the
+ * last dim, as mxfp4_quantize with along_rows = 0) and the token-dim codes
+ * (1x32 blocks along dim 0, output [cols, rows], as along_rows = 1).
+ *  in, groups, rows, cols, ld : as mxfp4_quantize.
+ *  row_params : the along-cols direction (along_rows must be 0, block 1x32).
+ *  col_params : the along-rows direction (along_rows must be 1, block 1x32).
+ *  Both directions use the same rounding and, for SR, the same sr_seed;
+ *  rht_d, rht_seed and sr_offset are per direction.
+ *  row_out, col_out : outputs of the two directions (codes_t/scales_mma_t
+ *  must be NULL).  Every output equals, bit for bit, what the two separate
+ *  mxfp4_quantize calls with these params write.
+ *  shapes : rows % 32 == 0 and cols % 32 == 0, else
+ *  MXFP4_ERR_UNSUPPORTED_SHAPE.
+ * Passage: the abstract (hybrid 1D/2D blocks: activations and gradients enter
+ * the forward/backward GEMMs along the contraction dim and the weight-gradient
+ * GEMM along the token dim, the latter with the RHT). */
+MXFP4_API mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, int64_t rows, int64_t cols,
+                                 int64_t ld, const mxfp4_quant_params* row_params,
+                                 const mxfp4_quant_params* col_params, const mxfp4_quant_outputs* row_out,
+                                 const mxfp4_quant_outputs* col_out, void* stream);
+
 /* Standalone randomized Hadamard transform along the last dim, d = 16:
  * out[r, :] = RHT(in[r, :]) in the butterfly order stated above.
  *  in  : device [rows, cols] (row stride ld elements), bf16 or f32.

@@ -78,3 +78,20 @@ def test_host_validation_without_gpu(libpath):
     d = mxfp4.DeoscParams(9, 0)
     assert L.mxfp4_deosc_update(ctypes.c_void_p(16), 1, 32, 32, 0, ctypes.byref(d), ctypes.c_void_p(16),
                                 ctypes.byref(o), None) == -1
+
+
+def test_dual_host_validation_without_gpu(libpath):
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    rp = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 0, 0, 0, 0, 0, 0)
+    cp = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0)
+    o = mxfp4.QuantOutputs(None, None, None, None, None)
+    args = lambda r, c: (None, 0, 1, 32, 32, 32, ctypes.byref(r), ctypes.byref(c), ctypes.byref(o), ctypes.byref(o),
+                         None)
+    assert L.mxfp4_quantize_dual(*args(rp, cp)) == -1                      # null input
+    assert L.mxfp4_quantize_dual(*args(cp, rp)) == -1                      # directions swapped
+    bad = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 1, 0, 0, mxfp4.ROUND_STOCHASTIC, 0, 0)
+    assert L.mxfp4_quantize_dual(*args(rp, bad)) == -1                     # rounding differs
+    assert L.mxfp4_quantize_dual(None, 0, 0, 32, 32, 32, ctypes.byref(rp), ctypes.byref(cp), ctypes.byref(o),
+                                 ctypes.byref(o), None) == 0                # empty: nothing to do
+
