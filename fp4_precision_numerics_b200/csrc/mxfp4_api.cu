@@ -452,6 +452,7 @@ mxfp4_status mxfp4_deosc_update(const float* master, int64_t groups, int64_t row
     if (!master || !state || !dp) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: null pointer");
     if (dp->flip_threshold < 1 || dp->flip_threshold > 7)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: flip_threshold must be in 1..7");
+    if (dp->freeze_lower > 1) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: freeze_lower must be 0 or 1");
     if (groups < 0 || rows < 0 || cols < 0) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_deosc_update: bad geometry");
     mxfp4_status s = check_outputs(out, true);
     if (s != MXFP4_OK) return s;
@@ -474,6 +475,7 @@ mxfp4_status mxfp4_deosc_update(const float* master, int64_t groups, int64_t row
     qa.step = step;
     qa.flip_threshold = dp->flip_threshold;
     qa.reset_period = dp->reset_period;
+    qa.freeze_lower = dp->freeze_lower;
     return launch_2d<float, true>(qa, false, false, static_cast<cudaStream_t>(stream));
 }
 

@@ -41,7 +41,7 @@ struct QuantArgs {
     uint8_t* scales_mma_t;            // 2D only
     // de-oscillation
     uint8_t* state;
-    uint32_t step, flip_threshold, reset_period;
+    uint32_t step, flip_threshold, reset_period, freeze_lower;
     // dual-direction quantisation: the 1x32-along-cols outputs of the same
     // input (codes [groups*rows, cols/2], scales, tensor-core scales)
     uint8_t* r_codes;
@@ -532,10 +532,20 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
                 c2 -= (c2 >> 3) & 0x01010101u;                                  // saturate 8 -> 7
                 const uint32_t updm = (upd >> 7) * 0xFFu;
                 const uint32_t frzm = (frz >> 7) * 0xFFu;
-                const uint32_t prev2 = (Q & updm) | (prev & ~updm);
+                uint32_t prev2 = (Q & updm) | (prev & ~updm);
                 const uint32_t frz2 = frz | (upd & ((c2 + thr_bias) & 0x80808080u));
-                s[2 * m + h] = prev2 | (c2 << 4) | frz2;
                 o[h] = (prev & frzm) | (Q & ~frzm);                             // frozen: stored code
+                if (a.freeze_lower) {
+                    // weights freezing now keep the lower-magnitude code of this
+                    // flip (magnitudes 0..7 per byte; ties keep Q)
+                    const uint32_t nfm = ((frz2 & ~frz) >> 7) * 0xFFu;
+                    const uint32_t mp = prev & 0x07070707u, mq = Q & 0x07070707u;
+                    const uint32_t ltm = ((((mq | 0x80808080u) - mp - 0x01010101u) & 0x80808080u) >> 7) * 0xFFu;
+                    const uint32_t keep = (prev & ltm) | (Q & ~ltm);           // prev where |prev| < |Q|
+                    prev2 = (keep & nfm) | (prev2 & ~nfm);
+                    o[h] = (keep & nfm) | (o[h] & ~nfm);
+                }
+                s[2 * m + h] = prev2 | (c2 << 4) | frz2;
             }
             w[m] = __byte_perm(o[0], o[1], 0x6420) | (__byte_perm(o[0], o[1], 0x7531) << 4);
         }

@@ -42,7 +42,8 @@ class QuantOutputs(ctypes.Structure):
 
 
 class DeoscParams(ctypes.Structure):
-    _fields_ = [("flip_threshold", ctypes.c_uint32), ("reset_period", ctypes.c_uint32)]
+    _fields_ = [("flip_threshold", ctypes.c_uint32), ("reset_period", ctypes.c_uint32),
+                ("freeze_lower", ctypes.c_uint32)]
 
 
 class Operand(ctypes.Structure):
@@ -252,7 +253,7 @@ def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, stream=None) -> tor
 
 def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_threshold: int = 4,
                  reset_period: int = 0, scales: bool = True, scales_mma: bool = False, transposed: bool = False,
-                 out: dict | None = None, stream=None) -> dict:
+                 out: dict | None = None, stream=None, freeze_lower: bool = False) -> dict:
     if master.dim() == 2:
         master = master.unsqueeze(0)
     assert master.dtype == torch.float32 and master.stride(-1) == 1
@@ -276,7 +277,8 @@ def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_thre
     outs = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")),
                         _ptr(o.get("codes_t")), _ptr(o.get("scales_mma_t")))
     mxfp4_deosc_update(ctypes.c_void_p(master.data_ptr()), G, R, C, int(step),
-                       DeoscParams(int(flip_threshold), int(reset_period)), ctypes.c_void_p(state.data_ptr()), outs,
+                       DeoscParams(int(flip_threshold), int(reset_period), int(bool(freeze_lower))),
+                       ctypes.c_void_p(state.data_ptr()), outs,
                        stream)
     return o
 

@@ -176,6 +176,10 @@ typedef struct {
     uint32_t flip_threshold; /* freeze once the flip count reaches this (default 4), 1..7 */
     uint32_t reset_period;   /* 0 = never; else clear counts and frozen bits on steps
                                 that are multiples of it */
+    uint32_t freeze_lower;   /* 0: a weight freezes at the code of its freezing flip
+                                (the new code).  1 (variant): it freezes at the
+                                lower-magnitude code of that flip (code & 7; ties
+                                keep the new code). */
 } mxfp4_deosc_params;
 
 /* Re-quantise fp32 master weights with 32x32 blocks and nearest rounding,
@@ -187,7 +191,9 @@ typedef struct {
  *    q = nearest code under the block scale of the current master weights;
  *    a frozen weight emits its stored code and keeps its state; otherwise,
  *    when q differs from the stored code the count increments, q is
- *    stored, and the weight freezes once count >= flip_threshold; it emits q.
+ *    stored, and the weight freezes once count >= flip_threshold; it emits q
+ *    (with freeze_lower, a weight freezing now stores and emits the
+ *    lower-magnitude of the old stored code and q instead).
  *  Scales always follow the current master weights.
  *  master: device f32 [groups, rows, cols]; state: device inout, same shape
  *  (one byte each).  out: codes [groups, rows, cols/2] plus any of the

@@ -79,7 +79,7 @@ def lib():
             L.oracle_quantize_1d_transposed.argtypes = qargs + [i64, ctypes.c_void_p, ctypes.c_void_p]
             L.oracle_quantize_2d.argtypes = qargs + [ctypes.c_void_p, ctypes.c_void_p]
             L.oracle_deosc_update.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_uint32, ctypes.c_uint32,
-                                              ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_uint32, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p,
                                               ctypes.c_void_p]
             L.oracle_dequant_1d.argtypes = [ctypes.c_void_p, ctypes.c_void_p, i64, i64, ctypes.c_void_p]
             L.oracle_dequant_2d.argtypes = [ctypes.c_void_p, ctypes.c_void_p, i64, i64, ctypes.c_void_p]
@@ -208,7 +208,7 @@ def quantize_2d(x: np.ndarray, rht_d: int = 0, rht_seed: int = 0, sr: bool = Fal
 
 
 def deosc_update(master: np.ndarray, step: int, state: np.ndarray, flip_threshold: int = 4,
-                 reset_period: int = 0):
+                 reset_period: int = 0, freeze_lower: bool = False):
     """One de-oscillation step over fp32 master weights [G, R, C].  Updates
     ``state`` in place; returns (codes [G, R, C/2], scales [G, R/32, C/32])."""
     master = np.ascontiguousarray(master, dtype=np.float32)
@@ -218,8 +218,8 @@ def deosc_update(master: np.ndarray, step: int, state: np.ndarray, flip_threshol
     assert state.dtype == np.uint8 and state.shape == (g, rows, cols) and state.flags["C_CONTIGUOUS"]
     codes = np.zeros((g, rows, cols // 2), dtype=np.uint8)
     scales = np.zeros((g, rows // 32, cols // 32), dtype=np.uint8)
-    lib().oracle_deosc_update(_ptr(master), g, rows, cols, step, flip_threshold, reset_period, _ptr(state),
-                              _ptr(codes), _ptr(scales))
+    lib().oracle_deosc_update(_ptr(master), g, rows, cols, step, flip_threshold, reset_period,
+                              int(bool(freeze_lower)), _ptr(state), _ptr(codes), _ptr(scales))
     return codes, scales
 
 

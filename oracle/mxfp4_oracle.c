@@ -441,13 +441,16 @@ void oracle_quantize_2d(const void* in, int dtype, int64_t rows, int64_t cols, i
 /*              the stored code, state unchanged.  Otherwise: if q differs   */
 /*              from the stored code, count = min(count+1, 7), store q, and  */
 /*              freeze once count >= flip_threshold; emit q.                 */
+/*  freeze_lower (variant): at the flip that freezes a weight, store and     */
+/*              emit the lower-magnitude of the two codes of that flip (the  */
+/*              stored one and q; magnitude = code & 7, ties keep q).        */
 /* Scales are always those of the current master weights (2D, 32x32).        */
 /* master: groups x rows x cols binary32; state/codes per weight;            */
 /* scales: groups x rows/32 x cols/32.                                       */
 /* ------------------------------------------------------------------------ */
 void oracle_deosc_update(const float* master, int64_t groups, int64_t rows, int64_t cols, uint32_t step,
-                         uint32_t flip_threshold, uint32_t reset_period, uint8_t* state, uint8_t* codes,
-                         uint8_t* scales)
+                         uint32_t flip_threshold, uint32_t reset_period, uint32_t freeze_lower, uint8_t* state,
+                         uint8_t* codes, uint8_t* scales)
 {
     int64_t per = rows * cols;
     int64_t nbr = rows / 32, nbc = cols / 32;
@@ -485,12 +488,19 @@ void oracle_deosc_update(const float* master, int64_t groups, int64_t rows, int6
                             if (frozen) {
                                 out = prev;
                             } else {
+                                out = q;
                                 if (q != prev) {
                                     count = count < 7 ? count + 1 : 7;
-                                    prev = q;
-                                    if ((uint32_t)count >= flip_threshold) frozen = 1;
+                                    int keep = q;
+                                    if ((uint32_t)count >= flip_threshold) {
+                                        frozen = 1;
+                                        /* variant: freeze to the lower-magnitude code of
+                                         * this flip (ties keep the new code) */
+                                        if (freeze_lower && (prev & 7) < (q & 7)) keep = prev;
+                                        out = keep;
+                                    }
+                                    prev = keep;
                                 }
-                                out = q;
                             }
                             st = (uint8_t)(prev | (count << 4) | (frozen << 7));
                         }

@@ -193,7 +193,8 @@ def test_rht_standalone():
 
 
 # ----------------------------------------------------------- de-oscillation
-def test_deosc_steps_bit_exact():
+@pytest.mark.parametrize("freeze_lower", [False, True])
+def test_deosc_steps_bit_exact(freeze_lower):
     G, R, C = 2, 256, 512
     w = synth.deosc_master(groups=G, rows=R, cols=C, seed=5)
     st_ref = np.zeros((G, R, C), dtype=np.uint8)
@@ -204,9 +205,11 @@ def test_deosc_steps_bit_exact():
             upd = synth.deosc_update_noise(w.shape, step, std=2e-4)
             w = (w + upd).astype(np.float32)
             wd.copy_(dev_f32(w))
-        out = mxfp4.deosc_update(wd, step, st, flip_threshold=4, reset_period=10, scales_mma=True, transposed=True)
+        out = mxfp4.deosc_update(wd, step, st, flip_threshold=4, reset_period=10, scales_mma=True, transposed=True,
+                                 freeze_lower=freeze_lower)
         torch.cuda.synchronize()
-        c_ref, s_ref = oracle.deosc_update(w, step, st_ref, flip_threshold=4, reset_period=10)
+        c_ref, s_ref = oracle.deosc_update(w, step, st_ref, flip_threshold=4, reset_period=10,
+                                           freeze_lower=freeze_lower)
         assert np.array_equal(host(st), st_ref), step
         assert np.array_equal(host(out["codes"]), c_ref), step
         assert np.array_equal(host(out["scales"]), s_ref), step

@@ -148,6 +148,33 @@ def test_deosc_frozen_code_follows_new_scale():
     assert scales[0, 0, 0] == 128 and (codes[0, 0, 0] & 0xF) == 2
 
 
+def test_deosc_freeze_lower_keeps_the_smaller_code():
+    """Variant: a weight alternating 1.3 / 1.2 (codes 3 <-> 2) freezes at its
+    4th flip (t = 4, new code 3, old code 2).  The default rule freezes the
+    new code 3; freeze_lower freezes 2, the lower magnitude, and emits it
+    from the freezing step on."""
+    seq = [1.3, 1.2, 1.3, 1.2, 1.3, 1.2, 1.3]
+    for lower, want_frozen in ((False, 3), (True, 2)):
+        st = np.zeros((1, 32, 32), dtype=np.uint8)
+        emitted = []
+        for t, v in enumerate(seq):
+            codes, _ = oracle.deosc_update(_block_with(v), t, st, flip_threshold=4, freeze_lower=lower)
+            emitted.append(int(codes[0, 0, 0] & 0x0F))
+        assert emitted == [3, 2, 3, 2, want_frozen, want_frozen, want_frozen]
+        assert (st[0, 0, 0] >> 7) == 1 and (st[0, 0, 0] & 0xF) == want_frozen
+
+
+def test_deosc_freeze_lower_tie_keeps_the_new_code():
+    """+-0.5 (codes 1 and 9) have equal magnitude: the new code is kept."""
+    st = np.zeros((1, 32, 32), dtype=np.uint8)
+    emitted = []
+    for t, v in enumerate([0.4, -0.4, 0.4, -0.4]):
+        codes, _ = oracle.deosc_update(_block_with(v), t, st, flip_threshold=2, freeze_lower=True)
+        emitted.append(int(codes[0, 0, 0] & 0x0F))
+    assert emitted == [1, 9, 1, 1]                       # freezes at t = 2 on the new code (+0.5)
+    assert (st[0, 0, 0] >> 7) == 1 and (st[0, 0, 0] & 0xF) == 1
+
+
 def test_dequant_closed_form():
     codes = np.array([[0x7F, 0x08]], dtype=np.uint8)           # codes 15, 7, 8, 0
     d = oracle.dequant_1d(np.tile(codes, (1, 8)), np.array([[130]], dtype=np.uint8))
