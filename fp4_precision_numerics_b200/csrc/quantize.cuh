@@ -637,6 +637,193 @@ __global__ void __launch_bounds__(kQ2dWarps * 32, 4) quant2d_kernel(QuantArgs a)
 }
 
 // ---------------------------------------------------------------------------
+// 2D 32x32 blocks with nearest rounding (weights), optionally with the
+// de-oscillation update, computed in the coalesced layout: lane l = 8 q + c
+// holds rows 4k + q (k = 0..7), elements 4c..4c+3 of its block, so every
+// load and store instruction of the warp covers 4 rows x 8 lanes of
+// contiguous bytes.  One 32-bit state word per row feeds the byte-parallel
+// de-oscillation update directly.  Codes leave as 16-bit pieces; the W^T
+// codes are built by an in-lane nibble transpose, a 4 x 4 word transpose
+// across the lanes 8 apart, and a second in-lane nibble transpose.
+// ---------------------------------------------------------------------------
+// Nibble-index bit swap on a 32-nibble vector in four 32-bit words (nibble
+// i = word i >> 3, position i & 7): exchanges index bits A < B, i.e. swaps
+// the nibbles at p and p + 2^B - 2^A for every p with bit A set and bit B
+// clear.  Bits 0-2 index inside a word, bits 3-4 the word.
+__host__ __device__ constexpr uint32_t nib_mask_pairs(int a, int b) {
+    uint32_t m = 0;
+    for (int n = 0; n < 8; ++n)
+        if (((n >> a) & 1) && !((n >> b) & 1)) m |= 0xFu << (4 * n);
+    return m;
+}
+
+__host__ __device__ constexpr uint32_t nib_mask_clear(int a) {
+    uint32_t m = 0;
+    for (int n = 0; n < 8; ++n)
+        if (!((n >> a) & 1)) m |= 0xFu << (4 * n);
+    return m;
+}
+
+template <int A, int B>
+__device__ __forceinline__ void nib_swap(uint32_t (&w)[4]) {
+    static_assert(A < B && B <= 4, "index bits");
+    if constexpr (B <= 2) {
+        constexpr int d = 4 * ((1 << B) - (1 << A));
+        constexpr uint32_t M = nib_mask_pairs(A, B);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t t = ((w[i] >> d) ^ w[i]) & M;
+            w[i] ^= t ^ (t << d);
+        }
+    } else if constexpr (A <= 2) {
+        constexpr int bb = B - 3, sh = 4 << A;
+        constexpr uint32_t M = nib_mask_clear(A);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if ((i >> bb) & 1) continue;
+            const int j = i + (1 << bb);
+            const uint32_t t = ((w[i] >> sh) ^ w[j]) & M;
+            w[j] ^= t;
+            w[i] ^= t << sh;
+        }
+    } else {
+        // both bits index the words (A = 3, B = 4): swap words 1 and 2
+        const uint32_t t = w[1];
+        w[1] = w[2];
+        w[2] = t;
+    }
+}
+
+template <typename InT, bool DEOSC>
+__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(QuantArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = lane >> 3, c = lane & 7;
+    const int64_t R = a.rows, C = a.cols;
+    const int64_t nbr = R >> 5, nbc = C >> 5;
+    const int64_t nblocks = a.groups * nbr * nbc;
+    const int64_t bid = int64_t(blockIdx.x) * kQ2dWarps + warp;
+    if (bid >= nblocks) return;
+    const int64_t g = bid / (nbr * nbc);
+    const int64_t rem = bid - g * nbr * nbc;
+    const int64_t bi = rem / nbc, bj = rem - bi * nbc;
+    const int64_t c0 = bj * 32;
+    const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
+    const int64_t row0 = g * R + bi * 32;   // global row of the block's row 0
+    float v[8][4];
+    uint32_t st[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int rr = 4 * k + q;
+        const InT* src = in + (bi * 32 + rr) * a.ld + c0 + 4 * c;
+        if constexpr (sizeof(InT) == 4) {
+            const float4 x = __ldg(reinterpret_cast<const float4*>(src));
+            v[k][0] = x.x; v[k][1] = x.y; v[k][2] = x.z; v[k][3] = x.w;
+        } else {
+            const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
+            v[k][0] = __uint_as_float(u.x << 16); v[k][1] = __uint_as_float(u.x & 0xFFFF0000u);
+            v[k][2] = __uint_as_float(u.y << 16); v[k][3] = __uint_as_float(u.y & 0xFFFF0000u);
+        }
+        if constexpr (DEOSC) st[k] = __ldg(reinterpret_cast<const uint32_t*>(a.state + (row0 + rr) * C + c0 + 4 * c));
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(v[k][j]));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    const int sb = scale_byte_from_amax(m);
+    const float inv = inv_scale_from_byte(sb);
+    uint32_t cw[8];   // codes of row 4k + q, elements 4c..4c+3 (nibble j = element 4c + j)
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        cw[k] = e2m1x2_rn(__fmul_rn(v[k][0], inv), __fmul_rn(v[k][1], inv)) |
+                (e2m1x2_rn(__fmul_rn(v[k][2], inv), __fmul_rn(v[k][3], inv)) << 8);
+    if constexpr (DEOSC) {
+        const bool reset = a.step > 0 && a.reset_period > 0 && (a.step % a.reset_period) == 0;
+        const uint32_t thr_bias = (0x80u - a.flip_threshold) * 0x01010101u;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            // the four codes spread to bytes (byte j = element 4c + j)
+            const uint32_t Q = __byte_perm(cw[k] & 0x0F0Fu, (cw[k] >> 4) & 0x0F0Fu, 0x5140);
+            uint32_t o;
+            if (a.step == 0) {
+                st[k] = Q;
+                o = Q;
+            } else {
+                const uint32_t S = st[k];
+                const uint32_t prev = S & 0x0F0F0F0Fu;
+                uint32_t cnt = (S >> 4) & 0x07070707u;
+                uint32_t frz = S & 0x80808080u;
+                if (reset) {
+                    cnt = 0u;
+                    frz = 0u;
+                }
+                const uint32_t ne = ((Q ^ prev) + 0x7F7F7F7Fu) & 0x80808080u;   // 0x80 where q != prev
+                const uint32_t upd = ne & ~frz;                                  // 0x80 where the weight flips
+                uint32_t c2 = cnt + (upd >> 7);
+                c2 -= (c2 >> 3) & 0x01010101u;                                   // saturate 8 -> 7
+                const uint32_t updm = (upd >> 7) * 0xFFu;
+                const uint32_t frzm = (frz >> 7) * 0xFFu;
+                uint32_t prev2 = (Q & updm) | (prev & ~updm);
+                const uint32_t frz2 = frz | (upd & ((c2 + thr_bias) & 0x80808080u));
+                o = (prev & frzm) | (Q & ~frzm);                                 // frozen: stored code
+                if (a.freeze_lower) {
+                    const uint32_t nfm = ((frz2 & ~frz) >> 7) * 0xFFu;
+                    const uint32_t mp = prev & 0x07070707u, mq = Q & 0x07070707u;
+                    const uint32_t ltm = ((((mq | 0x80808080u) - mp - 0x01010101u) & 0x80808080u) >> 7) * 0xFFu;
+                    const uint32_t keep = (prev & ltm) | (Q & ~ltm);
+                    prev2 = (keep & nfm) | (prev2 & ~nfm);
+                    o = (keep & nfm) | (o & ~nfm);
+                }
+                st[k] = prev2 | (c2 << 4) | frz2;
+            }
+            const uint32_t t = (o & 0x0F0F0F0Fu) | ((o & 0x0F0F0F0Fu) >> 4);   // byte 0: n0 n1, byte 2: n2 n3
+            cw[k] = __byte_perm(t, 0u, 0x4420) & 0xFFFFu;
+            *reinterpret_cast<uint32_t*>(a.state + (row0 + 4 * k + q) * C + c0 + 4 * c) = st[k];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        *reinterpret_cast<uint16_t*>(a.codes + (row0 + 4 * k + q) * (C >> 1) + (c0 >> 1) + 2 * c) = uint16_t(cw[k]);
+    if (a.scales && lane == 0) a.scales[g * nbr * nbc + bi * nbc + bj] = uint8_t(sb);
+    if (a.scales_mma) a.scales_mma[g * mma_scale_bytes(R, nbc) + mma_scale_offset(bi * 32 + lane, bj, nbc)] = uint8_t(sb);
+    if (a.codes_t) {
+        // rows 8 m .. 8 m + 7 of this lane's 8 x 4 code matrix (row k, column j) -> words
+        uint32_t w[4] = {cw[0] | (cw[1] << 16), cw[2] | (cw[3] << 16), cw[4] | (cw[5] << 16), cw[6] | (cw[7] << 16)};
+        // nibble 4k + j -> 8j + k: word j = column 4c + j over rows 4k + q
+        nib_swap<0, 2>(w);
+        nib_swap<1, 3>(w);
+        nib_swap<2, 4>(w);
+        nib_swap<3, 4>(w);
+        // lane (q, c) gathers column 4c + q from the lanes (q', c), q' = 0..3
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const bool up = lane & 16;
+            const uint32_t r = __shfl_xor_sync(0xFFFFFFFFu, up ? w[j] : w[j + 2], 16);
+            if (up) w[j] = r;
+            else w[j + 2] = r;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            const bool up = lane & 8;
+            const uint32_t r = __shfl_xor_sync(0xFFFFFFFFu, up ? w[j] : w[j + 1], 8);
+            if (up) w[j] = r;
+            else w[j + 1] = r;
+        }
+        // word q' = rows 4k + q' (nibble k) -> nibble 4k + q' = row-ordered W^T codes
+        nib_swap<0, 3>(w);
+        nib_swap<1, 4>(w);
+        nib_swap<2, 3>(w);
+        nib_swap<3, 4>(w);
+        const int64_t tr = g * C + c0 + 4 * c + q;   // row of W^T
+        *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + bi * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (a.scales_mma_t)
+            a.scales_mma_t[g * mma_scale_bytes(C, nbr) + mma_scale_offset(c0 + lane, bi, nbr)] = uint8_t(sb);
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Standalone RHT along the last dim: one thread per 16-element chunk.
 // ---------------------------------------------------------------------------
 template <typename InT, bool OUT_BF16>
