@@ -217,11 +217,12 @@ class Layer:
 # 8-expert / 4096-token layer, whose every tensor is exactly a quarter of the
 # full one, times 4.  An entry must go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": 4 * (664.1e6 + 244.8e6), "deosc_down": 4 * (332.1e6 + 107.2e6),
-    "dual_x": None, "dual_h": None, "dual_dy_up": None, "dual_dy_down": None,
-    "fprop_up": 4 * (97.5e6 + 336.1e6), "fprop_down": 4 * (61.3e6 + 141.0e6),
-    "dgrad_up": 4 * (122.5e6 + 153.2e6), "dgrad_down": 4 * (61.3e6 + 139.5e6),
-    "wgrad_up": 4 * (78.8e6 + 472.2e6), "wgrad_down": 4 * (51.9e6 + 205.9e6),
+    "deosc_up": 4 * (664.1e6 + 241.2e6), "deosc_down": 4 * (332.2e6 + 104.2e6),
+    "dual_x": 4 * (97.5e6 + 18.8e6), "dual_h": 4 * (97.5e6 + 16.0e6),
+    "dual_dy_up": 4 * (194.8e6 + 66.6e6), "dual_dy_down": 4 * (97.5e6 + 16.3e6),
+    "fprop_up": 4 * (97.5e6 + 333.4e6), "fprop_down": 4 * (61.3e6 + 139.1e6),
+    "dgrad_up": 4 * (122.5e6 + 153.3e6), "dgrad_down": 4 * (61.3e6 + 138.9e6),
+    "wgrad_up": 4 * (78.8e6 + 471.4e6), "wgrad_down": 4 * (52.0e6 + 205.8e6),
 }
 
 KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
