@@ -140,6 +140,39 @@ def test_wgrad_contracts_over_each_experts_tokens():
         assert comp <= TOL and norm <= TOL, (g, comp, norm)
 
 
+def test_more_than_255_groups_fprop_and_wgrad():
+    """300 groups: beyond the CTA-pair kernel's group table, so the call runs
+    the one-CTA kernel (128 x 192 tiles); empty and 1-3 tile groups."""
+    rng = np.random.default_rng(9)
+    seg = [int(v) * 128 for v in rng.choice([0, 1, 1, 2, 3], size=300)]
+    offs = np.concatenate([[0], np.cumsum(seg)])
+    M, N, K = int(offs[-1]), 224, 128
+    x = synth.bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    w = synth.bf16_bits((rng.standard_normal((len(seg), N, K)) * 0.02).astype(np.float32))
+    y, ref, ap = _fprop_case(x, w, offs)
+    comp, norm = gemm_errors(y, ref, ap)
+    assert comp <= TOL and norm <= TOL, (comp, norm)
+    # wgrad over the same 300 token groups
+    Nw, Kw = 96, 64
+    a = synth.bf16_bits(rng.standard_normal((M, Nw)).astype(np.float32))
+    b = synth.bf16_bits(rng.standard_normal((M, Kw)).astype(np.float32))
+    qa = mxfp4.quantize(dev_bf16(a), along_rows=True, scales=False, scales_mma=True)
+    qb = mxfp4.quantize(dev_bf16(b), along_rows=True, scales=False, scales_mma=True)
+    dw = host(mxfp4.grouped_gemm(mxfp4.GEMM_WGRAD, _offsets_dev(offs), qa["codes"], qa["scales_mma"], qb["codes"],
+                                 qb["scales_mma"], Nw, Kw, M))
+    mxfp4.mxfp4_check_device_status()
+    ca, sa = oracle.quantize_1d_transposed(a)
+    cb, sb = oracle.quantize_1d_transposed(b)
+    At, Bt = oracle.dequant_1d(ca, sa), oracle.dequant_1d(cb, sb)
+    for g in range(len(seg)):
+        lo, hi = int(offs[g]), int(offs[g + 1])
+        if hi == lo:
+            assert np.all(dw[g] == 0.0)
+            continue
+        comp, norm = gemm_errors(dw[g], At[:, lo:hi] @ Bt[:, lo:hi].T, np.abs(At[:, lo:hi]) @ np.abs(Bt[:, lo:hi]).T)
+        assert comp <= TOL and norm <= TOL, (g, comp, norm)
+
+
 def test_bad_group_offsets_flag_the_device_status():
     rng = np.random.default_rng(7)
     x = synth.bf16_bits(rng.standard_normal((256, 256)).astype(np.float32))
