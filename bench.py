@@ -140,6 +140,28 @@ class Layer:
             "wgrad_up": (F, D, M), "wgrad_down": (D, D, M),
         }
 
+    FUSED = ("fprop_up", "fprop_down", "dgrad_up", "dgrad_down")
+
+    def alloc_fused(self):
+        """Outputs of the fused-epilogue variant of the fprop/dgrad GEMMs:
+        bf16 Y and its 1x32-along-N codes and tensor-core scales."""
+        import torch
+        sb = self.mx.mxfp4_mma_scale_bytes
+        self.fused_out = {}
+        for name in self.FUSED:
+            Mg, N, _ = self.gemm_dims[name]
+            self.fused_out[name] = (torch.empty((Mg, N), dtype=torch.bfloat16, device=self.offsets.device),
+                                    dict(codes=torch.empty((Mg, N // 2), dtype=torch.uint8, device=self.offsets.device),
+                                         scales_mma=torch.empty((sb(Mg, N // 32),), dtype=torch.uint8,
+                                                                device=self.offsets.device)))
+
+    def fused_out_bytes(self, name):
+        """Algorithmic HBM bytes of one fused fprop/dgrad launch: operands read
+        once, bf16 output plus its codes and scales written once."""
+        Mg, N, K = self.gemm_dims[name]
+        per = 0.5 + 1.0 / 32
+        return (Mg * K + E * N * K) * per + Mg * N * (2 + per)
+
     def gemm_out_bytes(self, name):
         """Algorithmic HBM bytes of one GEMM launch: each operand's codes and
         scales read once, the binary32 output written once."""
@@ -149,11 +171,22 @@ class Layer:
             return (Mg + N) * K * per + E * Mg * N * 4
         return (Mg * K + E * N * K) * per + Mg * N * 4
 
-    def step(self, ev=None):
+    def step(self, ev=None, fused=False):
         """One training step.  `ev` (optional) maps a kernel name to a pair of
-        CUDA events recorded around its launch on the current stream."""
+        CUDA events recorded around its launch on the current stream.  With
+        `fused`, fprop and dgrad write bf16 outputs and their MXFP4
+        quantisation (the fused epilogue) instead of binary32."""
         mx = self.mx
         q = self.q
+
+        def gemm(name, op, a, b, b_codes, b_scales, Mg, N, K, out):
+            if fused:
+                y, qo = self.fused_out[name]
+                mx.grouped_gemm_fused(op, self.offsets, q[a]["codes"], q[a]["scales_mma"], q[b][b_codes],
+                                      q[b][b_scales], Mg, N, K, scales=False, y=y, out=qo)
+            else:
+                mx.grouped_gemm(op, self.offsets, q[a]["codes"], q[a]["scales_mma"], q[b][b_codes], q[b][b_scales],
+                                Mg, N, K, out=out)
 
         def rec(name, i):
             if ev is not None:
@@ -174,23 +207,20 @@ class Layer:
         mx.quantize_dual(self.x, col_rht_seed=1, scales=False, scales_mma=True, out_row=q["x"], out_col=q["xt"])
         rec("dual_x", 1)
         rec("fprop_up", 0)
-        mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["x"]["codes"], q["x"]["scales_mma"], q["w_up"]["codes"],
-                        q["w_up"]["scales_mma"], M, F, D, out=self.y_up)
+        gemm("fprop_up", mx.GEMM_FPROP, "x", "w_up", "codes", "scales_mma", M, F, D, self.y_up)
         rec("fprop_up", 1)
         rec("dual_h", 0)
         mx.quantize_dual(self.h, col_rht_seed=1, scales=False, scales_mma=True, out_row=q["h"], out_col=q["ht"])
         rec("dual_h", 1)
         rec("fprop_down", 0)
-        mx.grouped_gemm(mx.GEMM_FPROP, self.offsets, q["h"]["codes"], q["h"]["scales_mma"], q["w_down"]["codes"],
-                        q["w_down"]["scales_mma"], M, D, D, out=self.y_down)
+        gemm("fprop_down", mx.GEMM_FPROP, "h", "w_down", "codes", "scales_mma", M, D, D, self.y_down)
         rec("fprop_down", 1)
         rec("dual_dy_up", 0)
         mx.quantize_dual(self.dy_up, col_rht_seed=1, sr_seed=1, row_sr_offset=2 * s, col_sr_offset=1000 + 2 * s,
                          scales=False, scales_mma=True, out_row=q["dy_up"], out_col=q["dy_up_t"])
         rec("dual_dy_up", 1)
         rec("dgrad_up", 0)
-        mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_up"]["codes"], q["dy_up"]["scales_mma"],
-                        q["w_up"]["codes_t"], q["w_up"]["scales_mma_t"], M, D, F, out=self.dx)
+        gemm("dgrad_up", mx.GEMM_DGRAD, "dy_up", "w_up", "codes_t", "scales_mma_t", M, D, F, self.dx)
         rec("dgrad_up", 1)
         rec("dual_dy_down", 0)
         mx.quantize_dual(self.dy_down, col_rht_seed=1, sr_seed=1, row_sr_offset=2 * s + 1,
@@ -198,8 +228,7 @@ class Layer:
                          out_col=q["dy_down_t"])
         rec("dual_dy_down", 1)
         rec("dgrad_down", 0)
-        mx.grouped_gemm(mx.GEMM_DGRAD, self.offsets, q["dy_down"]["codes"], q["dy_down"]["scales_mma"],
-                        q["w_down"]["codes_t"], q["w_down"]["scales_mma_t"], M, D, D, out=self.dh)
+        gemm("dgrad_down", mx.GEMM_DGRAD, "dy_down", "w_down", "codes_t", "scales_mma_t", M, D, D, self.dh)
         rec("dgrad_down", 1)
         rec("wgrad_up", 0)
         mx.grouped_gemm(mx.GEMM_WGRAD, self.offsets, q["dy_up_t"]["codes"], q["dy_up_t"]["scales_mma"],
@@ -436,6 +465,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-steps", type=int, default=10,
+                    help="steps of the fused-epilogue variant timed after the main region (0: skip)")
     ap.add_argument("--experts", type=int, default=32,
                     help="smaller layers are for profiler captures only; the result line names the size")
     ap.add_argument("--tokens", type=int, default=16384)
@@ -523,6 +554,33 @@ def main():
             gbs = layer.quant_bytes[k] / (t / 1e3) / 1e9
             components[k] = {"ms": round(t, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
 
+    # ---------------- fused-epilogue variant (side measurement, not the step above)
+    # The same step with fprop/dgrad writing bf16 outputs plus their MXFP4
+    # quantisation straight from the accumulator instead of binary32.
+    fused = None
+    if args.fused_steps > 0:
+        layer.alloc_fused()
+        for _ in range(3):
+            layer.step(fused=True)
+        layer.mx.mxfp4_check_device_status()
+        fevs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
+                for _ in range(args.fused_steps)]
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.fused_steps):
+            layer.step(fevs[i], fused=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        layer.mx.mxfp4_check_device_status()
+        fk = {k: statistics.mean(e[k][0].elapsed_time(e[k][1]) for e in fevs) for k in layer.FUSED}
+        fused = {"steps": args.fused_steps, "ms_per_step": f0.elapsed_time(f1) / args.fused_steps,
+                 "kernels": {k: {"ms": round(fk[k], 4), "ms_binary32_out": round(per_kernel[k], 4),
+                                 "tflops": round(layer.gemm_flops[k] / (fk[k] / 1e3) / 1e12, 1),
+                                 "alg_gbs": round(layer.fused_out_bytes(k) / (fk[k] / 1e3) / 1e9, 1)}
+                             for k in layer.FUSED}}
+        del layer.fused_out
+
     # ---------------- end to end through the C ABI with host buffers
     # Every step uploads its inputs from pinned host memory and reads its
     # results back.  Two sets of device I/O buffers and three streams let the
@@ -606,6 +664,7 @@ def main():
         "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"], "reasons": ck["reasons"],
                    "samples": ck["samples"]},
         "cpu_baseline": cpu,
+        "fused_epilogue": fused,
     }
     if rank == 0:
         print(json.dumps(line))

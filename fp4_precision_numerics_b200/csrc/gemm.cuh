@@ -82,6 +82,11 @@ struct Args {
     int m_tiles, n_tiles;     // mode 0: over all rows of A; mode 1: per group
     int64_t total_tiles;
     uint32_t* status;
+    // fused epilogue (CTA-pair kernel, mode 0 only): bf16 output and its MXFP4
+    // quantisation in 1x32 blocks along N, in place of the binary32 output
+    // (bf16 [M][ldy] and codes [M][N/2] leave through tensor maps)
+    uint8_t* qscales;         // canonical [M][N/32], may be null
+    uint8_t* qscales_mma;     // tensor-core layout of the [M, N/32] scales, may be null
 };
 
 struct Tile {

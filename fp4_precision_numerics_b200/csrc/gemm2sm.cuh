@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "gemm.cuh"
+#include "quantize.cuh"
 
 namespace mxfp4 {
 namespace gemm2 {
@@ -48,6 +49,7 @@ constexpr uint32_t kBBytes = kSub * kBBox;
 constexpr uint32_t kSFABytes = kChunks * 512;    // chunks of 128 rows x 4 scales
 constexpr uint32_t kSFBBytes = 2 * kChunks * 512;  // two 128-row blocks of B
 constexpr uint32_t kEpiBufBytes = 32 * 32 * 4;
+constexpr uint32_t kEpiCodesOff = 32 * 32 * 2;   // fused epilogue: codes after the bf16 rows
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = BN;
 constexpr uint32_t kSfCol0 = 2 * kAccCols;       // 384
@@ -123,9 +125,15 @@ __device__ __forceinline__ Unit unit_info(const Args& a, const int32_t* s_off, c
     return un;
 }
 
+// FUSED (mode 0): the epilogue writes each output element as bf16 (round to
+// nearest even) and quantises every 32-column chunk of a row -- one lane's
+// registers -- as one 1x32 MXFP4 block of the bf16 values (nearest
+// rounding), i.e. exactly what mxfp4_quantize gives for the bf16 output.
+template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const __grid_constant__ CUtensorMap tmD, const Args a) {
+                            const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
+                            const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -165,6 +173,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmD);
+        if constexpr (FUSED) prefetch_tensormap(&tmQ);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -417,6 +426,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) r[i] = 0u;
                 }
                 if (!valid) continue;
+                if constexpr (FUSED) {
+                    // bf16 pairs (element 2i in the low half) and the block
+                    // maximum of the rounded values
+                    uint32_t hb[16];
+                    float m = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
+                            : "=r"(hb[i])
+                            : "f"(__uint_as_float(r[2 * i + 1])), "f"(__uint_as_float(r[2 * i])));
+                        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(hb[i] << 16)),
+                                           fabsf(__uint_as_float(hb[i] & 0xFFFF0000u))));
+                    }
+                    const int sbyte = scale_byte_from_amax(m);
+                    const float inv = inv_scale_from_byte(sbyte);
+                    uint32_t qb[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        qb[i >> 2] |= e2m1x2_rn(__fmul_rn(__uint_as_float(hb[i] << 16), inv),
+                                                __fmul_rn(__uint_as_float(hb[i] & 0xFFFF0000u), inv))
+                                      << (8 * (i & 3));
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
+                    // staging: 32 rows x 64 B of bf16 in the 64-byte swizzle
+                    // (16-byte chunk j of row r at chunk j ^ ((r >> 1) & 3)),
+                    // then 32 rows x 16 B of codes
+                    uint8_t* sbuf = stg + buf * kEpiBufBytes;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int pos = j ^ ((lane >> 1) & 3);
+                        *reinterpret_cast<uint4*>(sbuf + lane * 64 + pos * 16) =
+                            make_uint4(hb[4 * j], hb[4 * j + 1], hb[4 * j + 2], hb[4 * j + 3]);
+                    }
+                    *reinterpret_cast<uint4*>(sbuf + kEpiCodesOff + lane * 16) = make_uint4(qb[0], qb[1], qb[2], qb[3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    const int64_t col = un.n0 + 32 * c;
+                    if (lane == 0) {
+                        if (col < a.N && row < a.M) {   // N % 32 == 0: a chunk is all in or all out
+                            tma_store_2d(&tmD, sbuf, int32_t(col), int32_t(row));
+                            tma_store_2d(&tmQ, sbuf + kEpiCodesOff, int32_t(col >> 1), int32_t(row));
+                        }
+                        bulk_commit();
+                    }
+                    const int64_t grow = row + lane;
+                    if (grow < a.M && col < a.N) {
+                        const int64_t SN = a.N >> 5, s = col >> 5;
+                        if (a.qscales) a.qscales[grow * SN + s] = uint8_t(sbyte);
+                        if (a.qscales_mma) a.qscales_mma[mma_scale_offset(grow, s, SN)] = uint8_t(sbyte);
+                    }
+                    buf ^= 1u;
+                    continue;
+                }
                 if (lane == 0) bulk_wait_read<1>();
                 __syncwarp();
                 uint8_t* sb = stg + buf * kEpiBufBytes;

@@ -58,7 +58,8 @@ int pair_clusters() {
     cfg.gridDim = dim3(2 * unsigned(num_sms() / 2), 1, 1);
     cfg.blockDim = dim3(mxfp4::gemm2::kThreads, 1, 1);
     cfg.dynamicSmemBytes = mxfp4::gemm2::kSmemBytes;
-    if (cudaOccupancyMaxActiveClusters(&n, mxfp4::gemm2::grouped_gemm_2sm_kernel, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, mxfp4::gemm2::grouped_gemm_2sm_kernel<false>, &cfg) != cudaSuccess ||
+        n <= 0) {
         cudaGetLastError();
         n = num_sms() / 2;
     }
@@ -122,7 +123,8 @@ mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
 }
 
 bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box);
+                    const uint64_t* strides_bytes, const uint32_t* box,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE);
 
 template <typename InT>
 mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
@@ -252,7 +254,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
 }
 
 bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box) {
+                    const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t d[3], s[2];
@@ -263,8 +265,151 @@ bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void
     }
     for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
     return fn(m, dt, cuuint32_t(rank), const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FusedOut {
+    uint16_t* y;
+    int64_t ldy;
+    uint8_t* codes;
+    uint8_t* scales;
+    uint8_t* scales_mma;
+};
+
+// Shared by the binary32-output and the fused (bf16 + MXFP4) entry points:
+// argument checks, tensor maps, kernel choice and launch.  f != null selects
+// the fused epilogue of the CTA-pair kernel (out is then unused).
+mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offsets, mxfp4_operand A,
+                               mxfp4_operand B, int64_t M, int64_t N, int64_t K, float* out, int64_t ldo,
+                               const FusedOut* f, void* stream) {
+    using namespace mxfp4::gemm;
+    if (op != MXFP4_GEMM_FPROP && op != MXFP4_GEMM_DGRAD && op != MXFP4_GEMM_WGRAD)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad op %d", op);
+    if (num_groups <= 0 || !group_offsets || !A.codes || !A.scales_mma || !B.codes || !B.scales_mma)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: null pointer or num_groups <= 0");
+    if (M < 0 || N <= 0 || K < 0 || ldo < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad geometry");
+    if (num_groups > kMaxGroups)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: at most %d groups", kMaxGroups);
+    if (K % 128 && op == MXFP4_GEMM_WGRAD)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm(wgrad): total tokens must be a multiple of 128");
+    if (K % 64) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: K %% 64 != 0");
+    if (op != MXFP4_GEMM_WGRAD && M % 128)
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: M must be a multiple of 128 (padded groups)");
+    if (ldo % 4) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: ldo must be a multiple of 4");
+    if (!aligned16(A.codes) || !aligned16(B.codes) || !aligned16(A.scales_mma) || !aligned16(B.scales_mma) ||
+        (out && !aligned16(out)) || (reinterpret_cast<uintptr_t>(group_offsets) & 3u))
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: pointer not 16-byte aligned");
+    if (M == 0) return ok();
+    if (K == 0) {
+        if (op != MXFP4_GEMM_WGRAD) return ok();
+        // every group is empty: dW_g = 0
+        const cudaError_t e = cudaMemset2DAsync(out, size_t(ldo) * 4, 0, size_t(N) * 4, size_t(M) * num_groups,
+                                                static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: %s", cudaGetErrorString(e));
+        return ok();
+    }
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot resolve the device status word");
+
+    Args a{};
+    a.mode = op == MXFP4_GEMM_WGRAD ? 1 : 0;
+    a.num_groups = num_groups;
+    a.offsets = group_offsets;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.sfa = A.scales_mma;
+    a.sfb = B.scales_mma;
+    const int64_t S = (K + 31) / 32;
+    a.nchunk_a = (S + 3) / 4;
+    a.nchunk_b = (S + 3) / 4;
+    a.nrb_b = (N + 127) / 128;
+    a.sfb_group_bytes = mxfp4::mma_scale_bytes(N, S);
+    a.m_tiles = int((M + BM - 1) / BM);
+    a.n_tiles = int((N + BN - 1) / BN);
+    a.total_tiles = a.mode == 0 ? int64_t(a.m_tiles) * a.n_tiles : int64_t(num_groups) * a.m_tiles * a.n_tiles;
+    a.status = status;
+    if (f) {
+        a.qscales = f->scales;
+        a.qscales_mma = f->scales_mma;
+    }
+
+    const bool pair = pairs_enabled() && num_groups <= mxfp4::gemm2::kMaxGroups;
+    const uint32_t b_rows = pair ? uint32_t(mxfp4::gemm2::BNH) : uint32_t(BN);
+    CUtensorMap tmA, tmB, tmD, tmQ;
+    const uint64_t kb = uint64_t(K / 2);
+    {
+        const uint64_t dims[2] = {kb, uint64_t(M)};
+        const uint64_t str[1] = {kb};
+        const uint32_t box[2] = {128, BM};
+        if (!make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, A.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for A failed");
+    }
+    if (a.mode == 0) {
+        const uint64_t dims[3] = {kb, uint64_t(N), uint64_t(num_groups)};
+        const uint64_t str[2] = {kb, kb * uint64_t(N)};
+        const uint32_t box[3] = {128, b_rows, 1};
+        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, B.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
+        const uint64_t ddims[2] = {uint64_t(N), uint64_t(M)};
+        const uint64_t dstr[1] = {uint64_t(ldo) * 4};
+        const uint32_t dbox[2] = {32, 32};
+        if (f) {
+            // bf16 Y in 32 x 32 boxes (64-byte rows, 64-byte swizzle) and
+            // its codes in 32-row x 16-byte boxes
+            const uint64_t ydims[2] = {uint64_t(N), uint64_t(M)};
+            const uint64_t ystr[1] = {uint64_t(f->ldy) * 2};
+            const uint32_t ybox[2] = {32, 32};
+            if (!make_map_plain(&tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, f->y, ydims, ystr, ybox,
+                                CU_TENSOR_MAP_SWIZZLE_64B))
+                return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm_fused: tensor map for y failed");
+            const uint64_t qdims[2] = {uint64_t(N / 2), uint64_t(M)};
+            const uint64_t qstr[1] = {uint64_t(N / 2)};
+            const uint32_t qbox[2] = {16, 32};
+            if (!make_map_plain(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, f->codes, qdims, qstr, qbox))
+                return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm_fused: tensor map for codes failed");
+        } else if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, ddims, dstr, dbox)) {
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
+        }
+    } else {
+        const uint64_t dims[2] = {kb, uint64_t(N)};
+        const uint64_t str[1] = {kb};
+        const uint32_t box[2] = {128, b_rows};
+        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, B.codes, dims, str, box))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
+        const uint64_t ddims[3] = {uint64_t(N), uint64_t(M), uint64_t(num_groups)};
+        const uint64_t dstr[2] = {uint64_t(ldo) * 4, uint64_t(ldo) * 4 * uint64_t(M)};
+        const uint32_t dbox[3] = {32, 32, 1};
+        if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, ddims, dstr, dbox))
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
+    }
+    if (pair) {
+        namespace g2 = mxfp4::gemm2;
+        if (!f) tmQ = tmA;   // unused by the binary32 epilogue
+        void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const Args) =
+            f ? g2::grouped_gemm_2sm_kernel<true> : g2::grouped_gemm_2sm_kernel<false>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g2::kSmemBytes) != cudaSuccess)
+            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
+        // upper bound on the units (group, m-tile pair, n-tile): the exact
+        // count depends on the device-side offsets
+        const int64_t units = a.mode == 0 ? (int64_t(a.m_tiles) / 2 + num_groups) * a.n_tiles
+                                          : int64_t(num_groups) * ((a.m_tiles + 1) / 2) * a.n_tiles;
+        if (units == 0) return ok();
+        const int64_t clusters = pair_clusters();
+        const unsigned grid = 2u * unsigned(units < clusters ? units : clusters);
+        kern<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, tmQ, a);
+        return check_launch("mxfp4_grouped_gemm");
+    }
+    if (f) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: needs the CTA-pair kernel");
+    if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+        return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
+    if (a.total_tiles == 0) return ok();
+    const int64_t sms = num_sms();
+    const unsigned grid = unsigned(a.total_tiles < sms ? a.total_tiles : sms);
+    grouped_gemm_kernel<<<grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, a);
+    return check_launch("mxfp4_grouped_gemm");
 }
 
 }  // namespace
@@ -482,112 +627,29 @@ mxfp4_status mxfp4_deosc_update(const float* master, int64_t groups, int64_t row
 mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_offsets, mxfp4_operand A,
                                 mxfp4_operand B, int64_t M, int64_t N, int64_t K, float* out, int64_t ldo,
                                 void* stream) {
-    using namespace mxfp4::gemm;
-    if (op != MXFP4_GEMM_FPROP && op != MXFP4_GEMM_DGRAD && op != MXFP4_GEMM_WGRAD)
-        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad op %d", op);
-    if (num_groups <= 0 || !group_offsets || !A.codes || !A.scales_mma || !B.codes || !B.scales_mma || !out)
-        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: null pointer or num_groups <= 0");
-    if (M < 0 || N <= 0 || K < 0 || ldo < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: bad geometry");
-    if (num_groups > kMaxGroups)
-        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: at most %d groups", kMaxGroups);
-    if (K % 128 && op == MXFP4_GEMM_WGRAD)
-        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm(wgrad): total tokens must be a multiple of 128");
-    if (K % 64) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: K %% 64 != 0");
-    if (op != MXFP4_GEMM_WGRAD && M % 128)
-        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm: M must be a multiple of 128 (padded groups)");
-    if (ldo % 4) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: ldo must be a multiple of 4");
-    if (!aligned16(A.codes) || !aligned16(B.codes) || !aligned16(A.scales_mma) || !aligned16(B.scales_mma) ||
-        !aligned16(out) || (reinterpret_cast<uintptr_t>(group_offsets) & 3u))
-        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm: pointer not 16-byte aligned");
-    if (M == 0) return ok();
-    if (K == 0) {
-        if (op != MXFP4_GEMM_WGRAD) return ok();
-        // every group is empty: dW_g = 0
-        const cudaError_t e = cudaMemset2DAsync(out, size_t(ldo) * 4, 0, size_t(N) * 4, size_t(M) * num_groups,
-                                                static_cast<cudaStream_t>(stream));
-        if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: %s", cudaGetErrorString(e));
-        return ok();
-    }
-    uint32_t* status = status_word();
-    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot resolve the device status word");
+    if (!out) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm: null pointer or num_groups <= 0");
+    return grouped_gemm_impl(op, num_groups, group_offsets, A, B, M, N, K, out, ldo, nullptr, stream);
+}
 
-    Args a{};
-    a.mode = op == MXFP4_GEMM_WGRAD ? 1 : 0;
-    a.num_groups = num_groups;
-    a.offsets = group_offsets;
-    a.M = M;
-    a.N = N;
-    a.K = K;
-    a.sfa = A.scales_mma;
-    a.sfb = B.scales_mma;
-    const int64_t S = (K + 31) / 32;
-    a.nchunk_a = (S + 3) / 4;
-    a.nchunk_b = (S + 3) / 4;
-    a.nrb_b = (N + 127) / 128;
-    a.sfb_group_bytes = mxfp4::mma_scale_bytes(N, S);
-    a.m_tiles = int((M + BM - 1) / BM);
-    a.n_tiles = int((N + BN - 1) / BN);
-    a.total_tiles = a.mode == 0 ? int64_t(a.m_tiles) * a.n_tiles : int64_t(num_groups) * a.m_tiles * a.n_tiles;
-    a.status = status;
-
-    const bool pair = pairs_enabled() && num_groups <= mxfp4::gemm2::kMaxGroups;
-    const uint32_t b_rows = pair ? uint32_t(mxfp4::gemm2::BNH) : uint32_t(BN);
-    CUtensorMap tmA, tmB, tmD;
-    const uint64_t kb = uint64_t(K / 2);
-    {
-        const uint64_t dims[2] = {kb, uint64_t(M)};
-        const uint64_t str[1] = {kb};
-        const uint32_t box[2] = {128, BM};
-        if (!make_map(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, A.codes, dims, str, box))
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for A failed");
-    }
-    if (a.mode == 0) {
-        const uint64_t dims[3] = {kb, uint64_t(N), uint64_t(num_groups)};
-        const uint64_t str[2] = {kb, kb * uint64_t(N)};
-        const uint32_t box[3] = {128, b_rows, 1};
-        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, B.codes, dims, str, box))
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
-        const uint64_t ddims[2] = {uint64_t(N), uint64_t(M)};
-        const uint64_t dstr[1] = {uint64_t(ldo) * 4};
-        const uint32_t dbox[2] = {32, 32};
-        if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, out, ddims, dstr, dbox))
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
-    } else {
-        const uint64_t dims[2] = {kb, uint64_t(N)};
-        const uint64_t str[1] = {kb};
-        const uint32_t box[2] = {128, b_rows};
-        if (!make_map(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, B.codes, dims, str, box))
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B failed");
-        const uint64_t ddims[3] = {uint64_t(N), uint64_t(M), uint64_t(num_groups)};
-        const uint64_t dstr[2] = {uint64_t(ldo) * 4, uint64_t(ldo) * 4 * uint64_t(M)};
-        const uint32_t dbox[3] = {32, 32, 1};
-        if (!make_map(&tmD, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, ddims, dstr, dbox))
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D failed");
-    }
-    if (pair) {
-        namespace g2 = mxfp4::gemm2;
-        if (cudaFuncSetAttribute(g2::grouped_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 g2::kSmemBytes) != cudaSuccess)
-            return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
-        // upper bound on the units (group, m-tile pair, n-tile): the exact
-        // count depends on the device-side offsets
-        const int64_t units = a.mode == 0 ? (int64_t(a.m_tiles) / 2 + num_groups) * a.n_tiles
-                                          : int64_t(num_groups) * ((a.m_tiles + 1) / 2) * a.n_tiles;
-        if (units == 0) return ok();
-        const int64_t clusters = pair_clusters();
-        const unsigned grid = 2u * unsigned(units < clusters ? units : clusters);
-        g2::grouped_gemm_2sm_kernel<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(
-            tmA, tmB, tmD, a);
-        return check_launch("mxfp4_grouped_gemm");
-    }
-    if (cudaFuncSetAttribute(grouped_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
-        return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
-    if (a.total_tiles == 0) return ok();
-    const int64_t sms = num_sms();
-    const unsigned grid = unsigned(a.total_tiles < sms ? a.total_tiles : sms);
-    grouped_gemm_kernel<<<grid, kThreads, kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, a);
-    return check_launch("mxfp4_grouped_gemm");
+mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const int32_t* group_offsets, mxfp4_operand A,
+                                      mxfp4_operand B, int64_t M, int64_t N, int64_t K, uint16_t* y, int64_t ldy,
+                                      const mxfp4_quant_outputs* q, void* stream) {
+    if (op != MXFP4_GEMM_FPROP && op != MXFP4_GEMM_DGRAD)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: op must be FPROP or DGRAD");
+    if (!y || !q || !q->codes)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: null output pointer");
+    if (q->codes_t || q->scales_mma_t)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: codes_t / scales_mma_t are for 2D blocks only");
+    if (N % 32 || K <= 0) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: N %% 32 != 0 or K <= 0");
+    if (ldy < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: ldy < N");
+    if (ldy % 8) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm_fused: ldy must be a multiple of 8");
+    if (!aligned16(y) || !aligned16(q->codes))
+        return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm_fused: output pointer not 16-byte aligned");
+    if (num_groups > mxfp4::gemm2::kMaxGroups || !pairs_enabled())
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: at most %d groups, CTA pairs enabled",
+                    mxfp4::gemm2::kMaxGroups);
+    FusedOut f{y, ldy, q->codes, q->scales, q->scales_mma};
+    return grouped_gemm_impl(op, num_groups, group_offsets, A, B, M, N, K, nullptr, N, &f, stream);
 }
 
 }  // extern "C"

@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
             L.mxfp4_deosc_update.restype = st
             L.mxfp4_grouped_gemm.argtypes = [st, st, vp, Operand, Operand, i64, i64, i64, vp, i64, vp]
             L.mxfp4_grouped_gemm.restype = st
+            L.mxfp4_grouped_gemm_fused.argtypes = [st, st, vp, Operand, Operand, i64, i64, i64, vp, i64,
+                                                   ctypes.POINTER(QuantOutputs), vp]
+            L.mxfp4_grouped_gemm_fused.restype = st
             L.mxfp4_mma_scale_bytes.argtypes = [i64, i64]
             L.mxfp4_mma_scale_bytes.restype = ctypes.c_size_t
             L.mxfp4_last_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
@@ -155,6 +158,12 @@ def mxfp4_deosc_update(master_ptr, groups, rows, cols, step, params: DeoscParams
 
 def mxfp4_grouped_gemm(op, num_groups, offsets_ptr, a: Operand, b: Operand, M, N, K, out_ptr, ldo, stream=None):
     _check(lib().mxfp4_grouped_gemm(op, num_groups, offsets_ptr, a, b, M, N, K, out_ptr, ldo, _stream(stream)))
+
+
+def mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a: Operand, b: Operand, M, N, K, y_ptr, ldy,
+                             q: QuantOutputs, stream=None):
+    _check(lib().mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a, b, M, N, K, y_ptr, ldy, ctypes.byref(q),
+                                          _stream(stream)))
 
 
 def mxfp4_check_device_status(stream=None):
@@ -297,3 +306,30 @@ def grouped_gemm(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_codes,
                        Operand(b_codes.data_ptr(), b_scales_mma.data_ptr()), M, N, K,
                        ctypes.c_void_p(out.data_ptr()), ldo, stream)
     return out
+
+
+def grouped_gemm_fused(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_codes, b_scales_mma, M: int, N: int,
+                       K: int, scales: bool = True, scales_mma: bool = True, y: torch.Tensor | None = None,
+                       out: dict | None = None, stream=None) -> tuple:
+    """FPROP/DGRAD with the fused epilogue: returns (y, q) with y the [M, N]
+    bf16 output and q the dict ('codes', 'scales', 'scales_mma') of its
+    1x32-along-N MXFP4 quantisation with nearest rounding."""
+    assert offsets.dtype == torch.int32 and offsets.is_cuda
+    G = offsets.numel() - 1
+    dev = offsets.device
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    assert y.dtype == torch.bfloat16 and y.stride(-1) == 1
+    o = dict(out or {})
+    if "codes" not in o:
+        o["codes"] = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+    if scales and "scales" not in o:
+        o["scales"] = torch.empty((M, N // 32), dtype=torch.uint8, device=dev)
+    if scales_mma and "scales_mma" not in o:
+        o["scales_mma"] = torch.empty((mxfp4_mma_scale_bytes(M, N // 32),), dtype=torch.uint8, device=dev)
+    q = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")), None, None)
+    mxfp4_grouped_gemm_fused(op, G, ctypes.c_void_p(offsets.data_ptr()),
+                             Operand(a_codes.data_ptr(), a_scales_mma.data_ptr()),
+                             Operand(b_codes.data_ptr(), b_scales_mma.data_ptr()), M, N, K,
+                             ctypes.c_void_p(y.data_ptr()), y.stride(0), q, stream)
+    return y, o

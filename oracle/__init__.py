@@ -223,6 +223,21 @@ def deosc_update(master: np.ndarray, step: int, state: np.ndarray, flip_threshol
     return codes, scales
 
 
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Binary64 values -> bfloat16 bit patterns (uint16), rounded once to
+    nearest with ties to even: 8 significant bits, the binary32 exponent
+    range, spacing 2^-133 below 2^-126 (subnormals), and a result at or past
+    2^128 becomes infinity.  This is how a GEMM output is stored when the
+    next layer reads it as a bf16 activation (the recipe trains against a
+    BF16 baseline: abstract; roboaidigest "What ALTO Actually Does")."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)                        # |x| in [2^(e-1), 2^e)
+    q = np.maximum(e - 8, -133)               # exponent of one bf16 step at x
+    y = np.ldexp(np.round(np.ldexp(x, -q)), q)  # np.round: halves to even
+    y = np.where(np.abs(y) >= 2.0 ** 128, np.copysign(np.inf, x), y)
+    return (y.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
 def dequant_1d(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     codes = np.ascontiguousarray(codes)
     scales = np.ascontiguousarray(scales)

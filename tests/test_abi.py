@@ -95,3 +95,26 @@ def test_dual_host_validation_without_gpu(libpath):
     assert L.mxfp4_quantize_dual(None, 0, 0, 32, 32, 32, ctypes.byref(rp), ctypes.byref(cp), ctypes.byref(o),
                                  ctypes.byref(o), None) == 0                # empty: nothing to do
 
+
+
+def test_fused_gemm_host_validation_without_gpu(libpath):
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    a = mxfp4.Operand(16, 16)
+    q = mxfp4.QuantOutputs(16, None, None, None, None)
+    off, y = ctypes.c_void_p(16), ctypes.c_void_p(16)
+
+    def call(op=0, G=1, M=128, N=192, K=128, y=y, ldy=192, q=q):
+        return L.mxfp4_grouped_gemm_fused(op, G, off, a, a, M, N, K, y, ldy, ctypes.byref(q), None)
+
+    assert call(op=mxfp4.GEMM_WGRAD) == -1                                  # wgrad has no fused epilogue
+    assert call(y=None) == -1                                               # null y
+    assert call(N=200, ldy=200) == -2                                       # N % 32 != 0
+    assert call(K=0) == -2                                                  # nothing to contract
+    assert call(ldy=100) == -1                                              # ldy < N
+    assert call(ldy=196) == -3                                              # ldy % 8 != 0
+    assert call(y=ctypes.c_void_p(18)) == -3                                # misaligned y
+    assert call(G=300) == -2                                                # CTA-pair kernel only
+    assert call(q=mxfp4.QuantOutputs(16, None, None, 16, None)) == -1      # 2D-only outputs given
+    assert call(q=mxfp4.QuantOutputs(None, None, None, None, None)) == -1  # null codes
+    assert "fused" in mxfp4.last_error()

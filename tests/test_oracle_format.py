@@ -135,3 +135,42 @@ def test_rn_error_bound_on_tensor():
     sat = np.abs(v) > 6
     assert np.all(err[~sat] <= halfstep[~sat] + 1e-12)
     assert np.all(np.abs(deq[sat]) == 6 * scale[sat])
+
+
+# ---------------------------------------------------------------- bf16 output rounding
+def test_bf16_round_fixes_every_finite_bf16():
+    """Every finite bf16 value is already representable: it maps to itself."""
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = (bits.astype(np.uint32) << 16).view(np.float32)
+    keep = np.isfinite(vals)
+    assert np.array_equal(oracle.bf16_round(vals[keep].astype(np.float64)), bits[keep])
+
+
+def test_bf16_round_matches_torch_conversion_of_binary32():
+    """On binary32 inputs (exact in binary64) the rounding is torch's
+    float32 -> bfloat16 conversion: random bit patterns over the whole
+    exponent range, exact halfway cases of both parities, subnormals and the
+    overflow edge."""
+    import torch
+    rng = np.random.default_rng(17)
+    u = rng.integers(0, 1 << 32, size=200000, dtype=np.uint64).astype(np.uint32)
+    ties = (rng.integers(0, 1 << 16, size=20000, dtype=np.uint64).astype(np.uint32) << 16) | 0x8000
+    sub = rng.integers(0, 1 << 23, size=20000, dtype=np.uint64).astype(np.uint32)
+    edge = np.array([0x7F7F7FFF, 0x7F7F8000, 0x7F7FFFFF, 0x7F7F0000, 0x00000000, 0x80000000, 0x00008000,
+                     0x00018000, 0x3F808000, 0x3F818000], dtype=np.uint32)
+    u = np.concatenate([u, ties, sub, sub | 0x80000000, edge])
+    x = u.view(np.float32)
+    x = x[np.isfinite(x)]
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.bf16_round(x.astype(np.float64)), ref)
+
+
+def test_bf16_round_rounds_once_from_binary64():
+    """A binary64 value just above a bf16 halfway point rounds up, where a
+    detour through binary32 would land on the tie and round to even."""
+    t = 2.0 ** -30
+    cases = {1 + 2 ** -8 + t: 0x3F81, 1 + 2 ** -8: 0x3F80, 1 + 3 * 2 ** -8: 0x3F82, -(1 + 2 ** -8 + t): 0xBF81,
+             2.0 ** 128 - 2.0 ** 119: 0x7F80, 2.0 ** 128 - 2.0 ** 119 - 2.0 ** 100: 0x7F7F,
+             2.0 ** -134 + 2.0 ** -160: 0x0001, 2.0 ** -134: 0x0000}
+    got = oracle.bf16_round(np.array(list(cases), dtype=np.float64))
+    assert [int(g) for g in got] == list(cases.values())
