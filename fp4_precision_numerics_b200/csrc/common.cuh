@@ -110,6 +110,14 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     return d;
 }
 
+// max(|a|, |b|, |c|): the three-input form of max on sm_100 (one instruction
+// where two two-input maxima were needed).  Block maxima are built from it.
+__device__ __forceinline__ float fmax3_abs(float a, float b, float c) {
+    float d;
+    asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // ---------------------------------------------------------------------------
 // E2M1 conversions.
 // ---------------------------------------------------------------------------
@@ -123,6 +131,35 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
         : "=r"(out)
         : "f"(lo), "f"(hi));
     return out;
+}
+
+// Eight floats -> one word of eight E2M1 codes (nearest rounding as in
+// e2m1x2_rn), element k in bits 4k..4k+3: four conversions into byte
+// registers packed by one move.
+__device__ __forceinline__ uint32_t e2m1x8_rn(float e0, float e1, float e2, float e3, float e4, float e5, float e6,
+                                              float e7) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(e0), "f"(e1), "f"(e2), "f"(e3), "f"(e4), "f"(e5), "f"(e6), "f"(e7));
+    return out;
+}
+
+// Four floats -> 16 bits of E2M1 codes (nearest), element k in bits 4k..4k+3.
+__device__ __forceinline__ uint32_t e2m1x4_rn(float e0, float e1, float e2, float e3) {
+    uint16_t out;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b16 %0, {b0, b1};\n\t}"
+        : "=h"(out)
+        : "f"(e0), "f"(e1), "f"(e2), "f"(e3));
+    return uint32_t(out);
 }
 
 // Stochastic rounding of four values (already scaled into the block's range)

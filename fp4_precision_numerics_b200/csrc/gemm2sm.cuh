@@ -436,17 +436,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         asm("cvt.rn.bf16x2.f32 %0, %1, %2;"
                             : "=r"(hb[i])
                             : "f"(__uint_as_float(r[2 * i + 1])), "f"(__uint_as_float(r[2 * i])));
-                        m = fmaxf(m, fmaxf(fabsf(__uint_as_float(hb[i] << 16)),
-                                           fabsf(__uint_as_float(hb[i] & 0xFFFF0000u))));
+                        m = fmax3_abs(m, __uint_as_float(hb[i] << 16), __uint_as_float(hb[i] & 0xFFFF0000u));
                     }
                     const int sbyte = scale_byte_from_amax(m);
                     const float inv = inv_scale_from_byte(sbyte);
-                    uint32_t qb[4] = {0u, 0u, 0u, 0u};
+                    float y[32];   // scaled bf16 values in element order
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        qb[i >> 2] |= e2m1x2_rn(__fmul_rn(__uint_as_float(hb[i] << 16), inv),
-                                                __fmul_rn(__uint_as_float(hb[i] & 0xFFFF0000u), inv))
-                                      << (8 * (i & 3));
+                    for (int i = 0; i < 16; ++i) {
+                        y[2 * i] = __fmul_rn(__uint_as_float(hb[i] << 16), inv);
+                        y[2 * i + 1] = __fmul_rn(__uint_as_float(hb[i] & 0xFFFF0000u), inv);
+                    }
+                    uint32_t qb[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        qb[j] = e2m1x8_rn(y[8 * j], y[8 * j + 1], y[8 * j + 2], y[8 * j + 3], y[8 * j + 4],
+                                          y[8 * j + 5], y[8 * j + 6], y[8 * j + 7]);
                     if (lane == 0) bulk_wait_read<1>();
                     __syncwarp();
                     // staging: 32 rows x 64 B of bf16 in the 64-byte swizzle

@@ -46,6 +46,22 @@ int num_sms() {
     return n;
 }
 
+// CTAs of a persistent kernel that fit on the device at once (every SM
+// filled to its occupancy limit), cached per kernel; at least one per SM.
+template <typename K>
+int64_t resident_ctas(K kern, int threads, size_t smem) {
+    static int per_sm = 0;
+    if (per_sm <= 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 1;
+        }
+        per_sm = n;
+    }
+    return int64_t(num_sms()) * per_sm;
+}
+
 // Clusters of two CTAs of the pair GEMM that can be resident at once (one
 // CTA per SM; an SM left without a partner in its GPC stays idle).
 int pair_clusters() {
@@ -86,6 +102,14 @@ uint32_t* status_word() {
 
 // Host-side Philox4x32-10 (SC'11 constants) for the RHT sign word: bit i of
 // word 0 of Philox(key = seed, counter = (0, 0, 0, 1)).
+// (s_i / 4, s_i / 4) as two binary32 in one 64-bit word, for the packed RHT.
+void fill_rht_mul2(uint64_t (&m)[16], uint32_t signs) {
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t w = 0x3E800000u | (((signs >> i) & 1u) << 31);   // +-0.25
+        m[i] = w | (w << 32);
+    }
+}
+
 uint32_t rht_sign_mask(uint64_t seed) {
     uint32_t c[4] = {0u, 0u, 0u, 1u};
     uint32_t k0 = uint32_t(seed), k1 = uint32_t(seed >> 32);
@@ -129,6 +153,9 @@ bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void
 template <typename InT>
 mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
     // input [groups][rows = T][cols = F] with row stride ld: box = 128 features x (128 or 64) tokens
+    // the kernel indexes rows and features of all groups in 32 bits
+    if (qa.groups * qa.rows >= (int64_t(1) << 31) || qa.groups * qa.cols >= (int64_t(1) << 31))
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize: groups * rows and groups * cols must be < 2^31");
     CUtensorMap tm;
     const uint64_t esz = sizeof(InT);
     const uint64_t dims[3] = {uint64_t(qa.cols), uint64_t(qa.rows), uint64_t(qa.groups)};
@@ -141,12 +168,12 @@ mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
     if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_quantize: cannot resolve the device status word");
     const int64_t tt = mxfp4::cols_tt<InT>(), tf = mxfp4::kColsTF;
     const int64_t tiles = qa.groups * ((qa.rows + tt - 1) / tt) * ((qa.cols + tf - 1) / tf);
-    const int64_t cap = int64_t(num_sms()) * 4;
-    const unsigned grid = unsigned(tiles < cap ? tiles : cap);
     const uint32_t smem = mxfp4::cols_smem_bytes<InT>();
     auto go = [&](auto kern) -> mxfp4_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return fail(MXFP4_ERR_CUDA, "mxfp4_quantize(along rows): shared-memory attribute");
+        const int64_t cap = resident_ctas(kern, mxfp4::cols_threads<InT>(), smem);
+        const unsigned grid = unsigned(tiles < cap ? tiles : cap);
         kern<<<grid, mxfp4::cols_threads<InT>(), smem, st>>>(tm, qa, status);
         return check_launch("mxfp4_quantize(1d along rows)");
     };
@@ -158,6 +185,9 @@ mxfp4_status launch_cols(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
 
 template <typename InT>
 mxfp4_status launch_dual(const mxfp4::QuantArgs& qa, bool rht_col, bool rht_row, bool sr, cudaStream_t st) {
+    // the kernel indexes rows and features of all groups in 32 bits
+    if (qa.groups * qa.rows >= (int64_t(1) << 31) || qa.groups * qa.cols >= (int64_t(1) << 31))
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize: groups * rows and groups * cols must be < 2^31");
     CUtensorMap tm;
     const uint64_t esz = sizeof(InT);
     const uint64_t dims[3] = {uint64_t(qa.cols), uint64_t(qa.rows), uint64_t(qa.groups)};
@@ -170,12 +200,12 @@ mxfp4_status launch_dual(const mxfp4::QuantArgs& qa, bool rht_col, bool rht_row,
     if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_quantize_dual: cannot resolve the device status word");
     const int64_t tt = mxfp4::cols_tt<InT>(), tf = mxfp4::kColsTF;
     const int64_t tiles = qa.groups * ((qa.rows + tt - 1) / tt) * ((qa.cols + tf - 1) / tf);
-    const int64_t cap = int64_t(num_sms()) * 4;
-    const unsigned grid = unsigned(tiles < cap ? tiles : cap);
     const uint32_t smem = mxfp4::cols_smem_bytes<InT>();
     auto go = [&](auto kern) -> mxfp4_status {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return fail(MXFP4_ERR_CUDA, "mxfp4_quantize_dual: shared-memory attribute");
+        const int64_t cap = resident_ctas(kern, mxfp4::cols_threads<InT>(), smem);
+        const unsigned grid = unsigned(tiles < cap ? tiles : cap);
         kern<<<grid, mxfp4::cols_threads<InT>(), smem, st>>>(tm, qa, status);
         return check_launch("mxfp4_quantize_dual");
     };
@@ -488,6 +518,7 @@ mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_
     qa.cols = cols;
     qa.ld = ld;
     qa.rht_signs = p->rht_d == 16 ? rht_sign_mask(p->rht_seed) : 0u;
+    fill_rht_mul2(qa.rht_mul2, qa.rht_signs);
     qa.sr_key0 = uint32_t(p->sr_seed);
     qa.sr_key1 = uint32_t(p->sr_seed >> 32);
     qa.sr_offset = p->sr_offset;
@@ -545,6 +576,7 @@ mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, i
     qa.cols = cols;
     qa.ld = ld;
     qa.rht_signs = cp->rht_d == 16 ? rht_sign_mask(cp->rht_seed) : 0u;
+    fill_rht_mul2(qa.rht_mul2, qa.rht_signs);
     qa.sr_key0 = uint32_t(cp->sr_seed);
     qa.sr_key1 = uint32_t(cp->sr_seed >> 32);
     qa.sr_offset = cp->sr_offset;

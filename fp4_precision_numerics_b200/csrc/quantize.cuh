@@ -33,6 +33,7 @@ struct QuantArgs {
     const void* in;
     int64_t groups, rows, cols, ld;   // input geometry (per group: rows x cols, row stride ld)
     uint32_t rht_signs;               // bit i set -> sign i is -1 (only used with RHT)
+    uint64_t rht_mul2[16];            // packed (s_i / 4, s_i / 4): sign and 1/4 of RHT index i
     uint32_t sr_key0, sr_key1, sr_offset;
     uint8_t* codes;
     uint8_t* scales;                  // canonical, may be null
@@ -111,13 +112,11 @@ __device__ __forceinline__ void rht16(float (&x)[16], uint32_t signs) {
 // rht16 on two independent 16-element chunks at once, held as packed pairs
 // (chunk A in the low halves, chunk B in the high halves): every operation
 // is the scalar one of rht16 applied to both halves.
-__device__ __forceinline__ void rht16x2(uint64_t (&p)[16], uint32_t signs) {
-    const uint64_t quarter = f2_pack(0.25f, 0.25f);
+// `mul2[i]` holds s_i / 4 in both halves, so the sign and the 1/4 of index i
+// are one packed multiplication (s_i x / 4 is exactly (s_i x) * 1/4).
+__device__ __forceinline__ void rht16x2(uint64_t (&p)[16], const uint64_t (&mul2)[16]) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const uint64_t sbit = uint64_t((signs >> i) & 1u) << 31;
-        p[i] = f2_mul(p[i] ^ (sbit | (sbit << 32)), quarter);
-    }
+    for (int i = 0; i < 16; ++i) p[i] = f2_mul(p[i], mul2[i]);
 #pragma unroll
     for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
@@ -132,10 +131,10 @@ __device__ __forceinline__ void rht16x2(uint64_t (&p)[16], uint32_t signs) {
 }
 
 __device__ __forceinline__ float amax16(const float (&x)[16]) {
-    float m = 0.0f;
+    float m = fmax3_abs(x[0], x[1], x[2]);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(x[i]));
-    return m;
+    for (int i = 3; i < 15; i += 2) m = fmax3_abs(m, x[i], x[i + 1]);
+    return fmaxf(m, fabsf(x[15]));
 }
 
 // Scale 16 values by 2^-E and round them to 8 bytes of packed codes.
@@ -156,11 +155,8 @@ __device__ __forceinline__ uint2 quant16_scaled(const float (&v)[16], uint64_t n
         out.x = q0 | (q1 << 16);
         out.y = q2 | (q3 << 16);
     } else {
-        uint32_t b[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) b[i] = e2m1x2_rn(v[2 * i], v[2 * i + 1]);
-        out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-        out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+        out.x = e2m1x8_rn(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+        out.y = e2m1x8_rn(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
     }
     return out;
 }
@@ -169,8 +165,9 @@ template <bool SR>
 __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, uint64_t n0, const PhiloxKeys& keys,
                                          uint32_t offset) {
     float v[16];
+    const uint64_t inv2 = f2_pack(inv_scale, inv_scale);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(x[i], inv_scale);
+    for (int i = 0; i < 16; i += 2) f2_unpack(f2_mul(f2_pack(x[i], x[i + 1]), inv2), v[i], v[i + 1]);
     return quant16_scaled<SR>(v, n0, keys, offset);
 }
 
@@ -246,6 +243,48 @@ __host__ __device__ constexpr uint32_t cols_smem_bytes() { return kColsRing * co
 // features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
 // the input feeds both the contraction-dim codes and the token-dim codes.
 // Each thread takes two of the tile's (token row, 32-feature block) pairs.
+// Tile walk of a persistent CTA: tiles first, first + step, ... of a
+// [groups][token tiles][feature tiles] grid, kept as (g, tt, tf) and advanced
+// with adds and one conditional wrap per level (no division in the loop).
+struct TileWalk {
+    uint32_t g, tt, tf;
+    uint32_t sg, stt, stf;   // the step, decomposed the same way
+    uint32_t ntt, ntf;
+    __device__ void init(uint32_t t, uint32_t step, uint32_t ntt_, uint32_t ntf_) {
+        ntt = ntt_;
+        ntf = ntf_;
+        const uint32_t per = ntt * ntf;
+        g = t / per;
+        tt = (t - g * per) / ntf;
+        tf = t - g * per - tt * ntf;
+        sg = step / per;
+        stt = (step - sg * per) / ntf;
+        stf = step - sg * per - stt * ntf;
+    }
+    __device__ __forceinline__ void advance() {
+        tf += stf;
+        const uint32_t c1 = tf >= ntf ? 1u : 0u;
+        tf -= c1 * ntf;
+        tt += stt + c1;
+        const uint32_t c2 = tt >= ntt ? 1u : 0u;
+        tt -= c2 * ntt;
+        g += sg + c2;
+    }
+};
+
+// Byte offset of scale (r, s) in the tensor-core layout of one group whose
+// scale matrix has `nchunk` 4-scale chunks per row (32-bit form of
+// mma_scale_offset, for groups below 4 GB of scales).
+__device__ __forceinline__ uint32_t mma_off32(uint32_t r, uint32_t s, uint32_t nchunk) {
+    return ((r >> 7) * nchunk + (s >> 2)) * 512u + (r & 31u) * 16u + ((r >> 3) & 12u) + (s & 3u);
+}
+
+// Dual mode (DUAL): every tile is also quantised in 1x32 blocks along the
+// features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
+// the input feeds both the contraction-dim codes and the token-dim codes.
+// Each thread takes two of the tile's (token row, 32-feature block) pairs.
+// Indices are 32-bit (the host keeps groups * rows and groups * cols below
+// 2^31); products that address memory or count elements are widened.
 template <typename InT, bool RHT, bool SR, bool DUAL = false, bool RHT_R = false>
 __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
                                                            uint32_t* status) {
@@ -257,44 +296,45 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
     constexpr uint32_t kTile = cols_tile_bytes<InT>();
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kColsRing * kTile);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kColsRing * kTile + 8 * kColsRing);
-    const int64_t T = a.rows, F = a.cols;
-    const int64_t ntt = (T + kTT - 1) / kTT, ntf = (F + kTF - 1) / kTF;
-    const int64_t ntiles = a.groups * ntt * ntf;
-    const int64_t first = blockIdx.x;
-    const int64_t mine = first < ntiles ? (ntiles - first + gridDim.x - 1) / gridDim.x : 0;
-    auto tile_coords = [&](int64_t i, int64_t& g, int64_t& t0, int64_t& f0) {
-        const int64_t t = first + i * gridDim.x;
-        g = t / (ntt * ntf);
-        const int64_t r = t - g * ntt * ntf;
-        t0 = (r / ntf) * kTT;
-        f0 = (r - (r / ntf) * ntf) * kTF;
-    };
+    const uint32_t T = uint32_t(a.rows), F = uint32_t(a.cols);
+    const uint32_t ntt = (T + kTT - 1) / kTT, ntf = (F + kTF - 1) / kTF;
+    const uint32_t ntiles = uint32_t(a.groups) * ntt * ntf;
+    const uint32_t first = blockIdx.x, step = gridDim.x;
+    if (ntiles == 0) return;
+    const uint32_t mine = first < ntiles ? (ntiles - first + step - 1) / step : 0u;
     if (threadIdx.x == 0) {
         for (int b = 0; b < kColsRing; ++b) mbar_init(&full[b], 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_in);
-        for (int64_t i = 0; i < mine && i < kColsRing; ++i) {
-            int64_t g, t0, f0;
-            tile_coords(i, g, t0, f0);
+        TileWalk w;
+        w.init(first, step, ntt, ntf);
+        for (uint32_t i = 0; i < mine && i < uint32_t(kColsRing); ++i) {
             mbar_arrive_expect_tx(&full[i], kTile);
-            tma_load_3d(smem + i * kTile, &tm_in, &full[i], int32_t(f0), int32_t(t0), int32_t(g));
+            tma_load_3d(smem + i * kTile, &tm_in, &full[i], int32_t(w.tf * kTF), int32_t(w.tt * kTT), int32_t(w.g));
+            w.advance();
         }
     }
     __syncthreads();
+    TileWalk cur;                 // the tile being quantised
+    cur.init(first, step, ntt, ntf);
+    TileWalk nxt;                 // thread 0: the tile the freed buffer is refilled with
+    if (threadIdx.x == 0) nxt.init(first + uint32_t(kColsRing) * step, step, ntt, ntf);
     PhiloxKeys keys;
     if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
     const int pr = threadIdx.x % kPairs;   // features 2 pr, 2 pr + 1 of the tile
     const int blk = threadIdx.x / kPairs;  // 32-token block of the tile
-    const int64_t S = T >> 5;
-    for (int64_t i = 0; i < mine; ++i) {
+    const uint32_t S = T >> 5, SF = F >> 5;
+    const uint32_t nchunk_c = (S + 3) >> 2, nchunk_r = (SF + 3) >> 2;
+    const uint64_t mma_group_c = uint64_t((F + 127) >> 7) * nchunk_c * 512u;   // scale bytes of one group (col)
+    const uint64_t mma_group_r = uint64_t((T + 127) >> 7) * nchunk_r * 512u;   // (row direction)
+    for (uint32_t i = 0; i < mine; ++i) {
         const int b = int(i % kColsRing);
-        const uint32_t phase = uint32_t(i / kColsRing) & 1u;
+        const uint32_t phase = (i / kColsRing) & 1u;
         const bool got = mbar_wait_bounded(&full[b], phase, abort_flag, status, kRoleProducer);
-        int64_t g, t0, f0;
-        tile_coords(i, g, t0, f0);
-        const int64_t f = f0 + 2 * pr;
-        const int64_t tb = t0 + blk * 32;
+        const uint32_t g = cur.g, t0 = cur.tt * kTT, f0 = cur.tf * kTF;
+        const uint32_t f = f0 + 2 * pr;
+        const uint32_t tb = t0 + blk * 32;
         if (got && f < F && tb < T) {
             const uint8_t* tile = smem + b * kTile;   // [kTT][kTF] of InT, dense
             uint64_t p[32];                            // token k: (feature f, feature f + 1)
@@ -309,16 +349,17 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                 }
             }
             if constexpr (RHT) {
-                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[0]), a.rht_signs);
-                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[16]), a.rht_signs);
+                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[0]), a.rht_mul2);
+                rht16x2(*reinterpret_cast<uint64_t(*)[16]>(&p[16]), a.rht_mul2);
             }
             float m0 = 0.0f, m1 = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 32; ++k) {
-                float lo, hi;
-                f2_unpack(p[k], lo, hi);
-                m0 = fmaxf(m0, fabsf(lo));
-                m1 = fmaxf(m1, fabsf(hi));
+            for (int k = 0; k < 32; k += 2) {
+                float lo0, hi0, lo1, hi1;
+                f2_unpack(p[k], lo0, hi0);
+                f2_unpack(p[k + 1], lo1, hi1);
+                m0 = fmax3_abs(m0, lo0, lo1);
+                m1 = fmax3_abs(m1, hi0, hi1);
             }
             const int sb0 = scale_byte_from_amax(m0), sb1 = scale_byte_from_amax(m1);
             const uint64_t inv = f2_pack(inv_scale_from_byte(sb0), inv_scale_from_byte(sb1));
@@ -326,33 +367,31 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
 #pragma unroll
             for (int k = 0; k < 32; ++k) f2_unpack(f2_mul(p[k], inv), v0[k], v1[k]);
             const bool two = f + 1 < F;
-            const int64_t orow = g * F + f;  // output row of feature f (groups back to back)
-            const int64_t s = tb >> 5;
+            const uint32_t orow = g * F + f;   // output row of feature f (groups back to back)
+            const uint32_t s = tb >> 5;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 if (h == 1 && !two) break;
                 const float* v = h ? v1 : v0;
-                const uint64_t n0 = uint64_t(orow + h) * uint64_t(T) + uint64_t(tb);
+                const uint64_t n0 = uint64_t(orow + h) * T + tb;
                 const uint2 q0 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v), n0, keys, a.sr_offset);
                 const uint2 q1 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v + 16), n0 + 16, keys,
                                                     a.sr_offset);
-                *reinterpret_cast<uint4*>(a.codes + (orow + h) * (T >> 1) + (tb >> 1)) =
+                *reinterpret_cast<uint4*>(a.codes + uint64_t(orow + h) * (T >> 1) + (tb >> 1)) =
                     make_uint4(q0.x, q0.y, q1.x, q1.y);
                 const int sb = h ? sb1 : sb0;
-                if (a.scales) a.scales[(orow + h) * S + s] = uint8_t(sb);
-                if (a.scales_mma)
-                    a.scales_mma[g * mma_scale_bytes(F, S) + mma_scale_offset(f + h, s, S)] = uint8_t(sb);
+                if (a.scales) a.scales[uint64_t(orow + h) * S + s] = uint8_t(sb);
+                if (a.scales_mma) a.scales_mma[g * mma_group_c + mma_off32(f + h, s, nchunk_c)] = uint8_t(sb);
             }
         }
         if constexpr (DUAL) {
             // the same tile, 1x32 blocks along the features
             constexpr int kChunks16 = 32 * int(sizeof(InT)) / 16;   // 16-byte chunks per 32-element block
-            const int64_t SF = F >> 5;
             const uint8_t* tile = smem + b * kTile;
 #pragma unroll 1
             for (int e = threadIdx.x; e < kTT * (kTF / 32); e += blockDim.x) {
                 const int rr = e / (kTF / 32), fb = e % (kTF / 32);
-                const int64_t t = t0 + rr, fc = f0 + 32 * fb;
+                const uint32_t t = t0 + rr, fc = f0 + 32 * fb;
                 if (!got || t >= T || fc >= F) continue;
                 const uint8_t* src = tile + (rr * kTF + 32 * fb) * int(sizeof(InT));
                 // bf16: a block is 4 chunks of 16 bytes and half a 128-byte bank
@@ -364,56 +403,131 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                 const int m = sizeof(InT) == 2 ? (((fb >> 1) | ((rr & 1) << 1)) & 3) : 0;
 #pragma unroll
                 for (int j = 0; j < kChunks16; ++j) w[j] = *reinterpret_cast<const uint4*>(src + 16 * (j ^ m));
-                if constexpr (sizeof(InT) == 2) {
-                    if (m & 1) {
-                        const uint4 t01 = w[0], t23 = w[2];
-                        w[0] = w[1]; w[1] = t01; w[2] = w[3]; w[3] = t23;
-                    }
-                    if (m & 2) {
-                        const uint4 t0 = w[0], t1 = w[1];
-                        w[0] = w[2]; w[1] = w[3]; w[2] = t0; w[3] = t1;
-                    }
-                }
-                float x[32];
+                const uint32_t row = g * T + t;   // output row (groups back to back)
+                const uint64_t n0 = uint64_t(row) * F + fc;
+                int sb;
+                uint32_t cw[4];                   // codes of elements 8j .. 8j + 7
+                if constexpr (sizeof(InT) == 2 && !RHT_R) {
+                    // Slot j holds chunk j ^ m.  The block maximum and the
+                    // scaling do not depend on the order, so the data stay
+                    // in slot order and only the four code words (and, for
+                    // SR, the chunks' random words) are permuted.
+                    float x[32];
 #pragma unroll
-                for (int j = 0; j < kChunks16; ++j) {
-                    const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
-                    if constexpr (sizeof(InT) == 2) {
+                    for (int j = 0; j < 4; ++j) {
+                        const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             x[8 * j + 2 * q] = __uint_as_float(ww[q] << 16);
                             x[8 * j + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
                         }
+                    }
+                    sb = scale_byte_from_amax(fmaxf(amax16(*reinterpret_cast<float(*)[16]>(&x[0])),
+                                                    amax16(*reinterpret_cast<float(*)[16]>(&x[16]))));
+                    const uint64_t inv2 = f2_pack(inv_scale_from_byte(sb), inv_scale_from_byte(sb));
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) f2_unpack(f2_mul(f2_pack(x[i], x[i + 1]), inv2), v[i], v[i + 1]);
+                    if constexpr (SR) {
+                        // chunk c takes words 2c, 2c + 1 of the block's two
+                        // Philox calls (elements 0-15 and 16-31)
+                        const uint64_t gq = n0 >> 4;
+                        const Philox4 r0 = philox4x32_10(uint32_t(gq), uint32_t(gq >> 32), a.r_sr_offset, 0u, keys);
+                        const Philox4 r1 =
+                            philox4x32_10(uint32_t(gq + 1), uint32_t((gq + 1) >> 32), a.r_sr_offset, 0u, keys);
+                        uint32_t R[8] = {r0.w[0], r0.w[1], r0.w[2], r0.w[3], r1.w[0], r1.w[1], r1.w[2], r1.w[3]};
+                        if (m & 1) {
+                            uint32_t tq;
+                            tq = R[0]; R[0] = R[2]; R[2] = tq;
+                            tq = R[1]; R[1] = R[3]; R[3] = tq;
+                            tq = R[4]; R[4] = R[6]; R[6] = tq;
+                            tq = R[5]; R[5] = R[7]; R[7] = tq;
+                        }
+                        if (m & 2) {
+                            uint32_t tq;
+                            tq = R[0]; R[0] = R[4]; R[4] = tq;
+                            tq = R[1]; R[1] = R[5]; R[5] = tq;
+                            tq = R[2]; R[2] = R[6]; R[6] = tq;
+                            tq = R[3]; R[3] = R[7]; R[7] = tq;
+                        }
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            cw[j] = e2m1x4_sr(v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3], R[2 * j]) |
+                                    (e2m1x4_sr(v[8 * j + 4], v[8 * j + 5], v[8 * j + 6], v[8 * j + 7], R[2 * j + 1])
+                                     << 16);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) x[4 * j + q] = __uint_as_float(ww[q]);
+                        for (int j = 0; j < 4; ++j)
+                            cw[j] = e2m1x8_rn(v[8 * j], v[8 * j + 1], v[8 * j + 2], v[8 * j + 3], v[8 * j + 4],
+                                              v[8 * j + 5], v[8 * j + 6], v[8 * j + 7]);
                     }
+                    // chunk c's codes sit in cw[c ^ m]
+                    if (m & 1) {
+                        uint32_t tq;
+                        tq = cw[0]; cw[0] = cw[1]; cw[1] = tq;
+                        tq = cw[2]; cw[2] = cw[3]; cw[3] = tq;
+                    }
+                    if (m & 2) {
+                        uint32_t tq;
+                        tq = cw[0]; cw[0] = cw[2]; cw[2] = tq;
+                        tq = cw[1]; cw[1] = cw[3]; cw[3] = tq;
+                    }
+                } else {
+                    if constexpr (sizeof(InT) == 2) {
+                        if (m & 1) {
+                            const uint4 t01 = w[0], t23 = w[2];
+                            w[0] = w[1]; w[1] = t01; w[2] = w[3]; w[3] = t23;
+                        }
+                        if (m & 2) {
+                            const uint4 tq0 = w[0], tq1 = w[1];
+                            w[0] = w[2]; w[1] = w[3]; w[2] = tq0; w[3] = tq1;
+                        }
+                    }
+                    float x[32];
+#pragma unroll
+                    for (int j = 0; j < kChunks16; ++j) {
+                        const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+                        if constexpr (sizeof(InT) == 2) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                x[8 * j + 2 * q] = __uint_as_float(ww[q] << 16);
+                                x[8 * j + 2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) x[4 * j + q] = __uint_as_float(ww[q]);
+                        }
+                    }
+                    float (&x0)[16] = *reinterpret_cast<float(*)[16]>(&x[0]);
+                    float (&x1)[16] = *reinterpret_cast<float(*)[16]>(&x[16]);
+                    if constexpr (RHT_R) {
+                        rht16(x0, a.r_rht_signs);
+                        rht16(x1, a.r_rht_signs);
+                    }
+                    sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
+                    const float inv = inv_scale_from_byte(sb);
+                    const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.r_sr_offset);
+                    const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.r_sr_offset);
+                    cw[0] = q0.x;
+                    cw[1] = q0.y;
+                    cw[2] = q1.x;
+                    cw[3] = q1.y;
                 }
-                float (&x0)[16] = *reinterpret_cast<float(*)[16]>(&x[0]);
-                float (&x1)[16] = *reinterpret_cast<float(*)[16]>(&x[16]);
-                if constexpr (RHT_R) {
-                    rht16(x0, a.r_rht_signs);
-                    rht16(x1, a.r_rht_signs);
-                }
-                const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
-                const float inv = inv_scale_from_byte(sb);
-                const int64_t row = g * T + t;   // output row (groups back to back)
-                const uint64_t n0 = uint64_t(row) * uint64_t(F) + uint64_t(fc);
-                const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.r_sr_offset);
-                const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.r_sr_offset);
-                *reinterpret_cast<uint4*>(a.r_codes + row * (F >> 1) + (fc >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
-                const int64_t s = fc >> 5;
-                if (a.r_scales) a.r_scales[row * SF + s] = uint8_t(sb);
-                if (a.r_scales_mma) a.r_scales_mma[g * mma_scale_bytes(T, SF) + mma_scale_offset(t, s, SF)] = uint8_t(sb);
+                *reinterpret_cast<uint4*>(a.r_codes + uint64_t(row) * (F >> 1) + (fc >> 1)) =
+                    make_uint4(cw[0], cw[1], cw[2], cw[3]);
+                const uint32_t sc = fc >> 5;
+                if (a.r_scales) a.r_scales[uint64_t(row) * SF + sc] = uint8_t(sb);
+                if (a.r_scales_mma) a.r_scales_mma[g * mma_group_r + mma_off32(t, sc, nchunk_r)] = uint8_t(sb);
             }
         }
         __syncthreads();  // buffer b fully read: refill it with tile i + kColsRing
         if (threadIdx.x == 0 && i + kColsRing < mine) {
-            int64_t g2, t2, f2;
-            tile_coords(i + kColsRing, g2, t2, f2);
             mbar_arrive_expect_tx(&full[b], kTile);
-            tma_load_3d(smem + b * kTile, &tm_in, &full[b], int32_t(f2), int32_t(t2), int32_t(g2));
+            tma_load_3d(smem + b * kTile, &tm_in, &full[b], int32_t(nxt.tf * kTF), int32_t(nxt.tt * kTT),
+                        int32_t(nxt.g));
+            nxt.advance();
         }
+        cur.advance();
     }
 }
 
@@ -727,9 +841,7 @@ __global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(QuantArgs 
     }
     float m = 0.0f;
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(v[k][j]));
+    for (int k = 0; k < 8; ++k) m = fmax3_abs(fmax3_abs(m, v[k][0], v[k][1]), v[k][2], v[k][3]);
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     const int sb = scale_byte_from_amax(m);
@@ -737,8 +849,8 @@ __global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(QuantArgs 
     uint32_t cw[8];   // codes of row 4k + q, elements 4c..4c+3 (nibble j = element 4c + j)
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-        cw[k] = e2m1x2_rn(__fmul_rn(v[k][0], inv), __fmul_rn(v[k][1], inv)) |
-                (e2m1x2_rn(__fmul_rn(v[k][2], inv), __fmul_rn(v[k][3], inv)) << 8);
+        cw[k] = e2m1x4_rn(__fmul_rn(v[k][0], inv), __fmul_rn(v[k][1], inv), __fmul_rn(v[k][2], inv),
+                          __fmul_rn(v[k][3], inv));
     if constexpr (DEOSC) {
         const bool reset = a.step > 0 && a.reset_period > 0 && (a.step % a.reset_period) == 0;
         const uint32_t thr_bias = (0x80u - a.flip_threshold) * 0x01010101u;
