@@ -44,7 +44,7 @@ struct PhiloxKeys {
     uint32_t k0[10], k1[10];
 };
 
-__device__ __forceinline__ PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
+__host__ __device__ __forceinline__ PhiloxKeys philox_keys(uint32_t k0, uint32_t k1) {
     PhiloxKeys k;
 #pragma unroll
     for (int r = 0; r < 10; ++r) {

@@ -520,6 +520,7 @@ mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t groups, int64_
     qa.rht_signs = p->rht_d == 16 ? rht_sign_mask(p->rht_seed) : 0u;
     fill_rht_mul2(qa.rht_mul2, qa.rht_signs);
     qa.sr_key0 = uint32_t(p->sr_seed);
+    qa.sr_keys = mxfp4::philox_keys(uint32_t(p->sr_seed), uint32_t(p->sr_seed >> 32));
     qa.sr_key1 = uint32_t(p->sr_seed >> 32);
     qa.sr_offset = p->sr_offset;
     qa.codes = out->codes;
@@ -578,6 +579,7 @@ mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, i
     qa.rht_signs = cp->rht_d == 16 ? rht_sign_mask(cp->rht_seed) : 0u;
     fill_rht_mul2(qa.rht_mul2, qa.rht_signs);
     qa.sr_key0 = uint32_t(cp->sr_seed);
+    qa.sr_keys = mxfp4::philox_keys(uint32_t(cp->sr_seed), uint32_t(cp->sr_seed >> 32));
     qa.sr_key1 = uint32_t(cp->sr_seed >> 32);
     qa.sr_offset = cp->sr_offset;
     qa.codes = col_out->codes;

@@ -35,6 +35,7 @@ struct QuantArgs {
     uint32_t rht_signs;               // bit i set -> sign i is -1 (only used with RHT)
     uint64_t rht_mul2[16];            // packed (s_i / 4, s_i / 4): sign and 1/4 of RHT index i
     uint32_t sr_key0, sr_key1, sr_offset;
+    PhiloxKeys sr_keys;               // the ten round keys of (sr_key0, sr_key1), filled by the host
     uint8_t* codes;
     uint8_t* scales;                  // canonical, may be null
     uint8_t* scales_mma;              // tensor-core layout, may be null
@@ -179,15 +180,14 @@ __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, 
 // (groups back to back).
 // ---------------------------------------------------------------------------
 template <typename InT, bool RHT, bool SR>
-__global__ void __launch_bounds__(256) quant1d_rows_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(256) quant1d_rows_kernel(const __grid_constant__ QuantArgs a) {
     const int64_t C = a.cols;
     const int64_t S = C >> 5;
     const int64_t total = a.groups * a.rows * S;
     const int64_t mma_group_bytes = mma_scale_bytes(a.rows, S);
     const InT* in = static_cast<const InT*>(a.in);
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
-    PhiloxKeys keys;
-    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
+    const PhiloxKeys& keys = a.sr_keys;   // kernel parameters: read from the constant bank
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
         const int64_t row = i / S;
         const int64_t s = i - row * S;
@@ -286,7 +286,7 @@ __device__ __forceinline__ uint32_t mma_off32(uint32_t r, uint32_t s, uint32_t n
 // Indices are 32-bit (the host keeps groups * rows and groups * cols below
 // 2^31); products that address memory or count elements are widened.
 template <typename InT, bool RHT, bool SR, bool DUAL = false, bool RHT_R = false>
-__global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, QuantArgs a,
+__global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_constant__ CUtensorMap tm_in, const __grid_constant__ QuantArgs a,
                                                            uint32_t* status) {
     constexpr int kTT = cols_tt<InT>();
     constexpr int kTF = kColsTF;
@@ -320,8 +320,7 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
     cur.init(first, step, ntt, ntf);
     TileWalk nxt;                 // thread 0: the tile the freed buffer is refilled with
     if (threadIdx.x == 0) nxt.init(first + uint32_t(kColsRing) * step, step, ntt, ntf);
-    PhiloxKeys keys;
-    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
+    const PhiloxKeys& keys = a.sr_keys;   // kernel parameters: read from the constant bank
     const int pr = threadIdx.x % kPairs;   // features 2 pr, 2 pr + 1 of the tile
     const int blk = threadIdx.x / kPairs;  // 32-token block of the tile
     const uint32_t S = T >> 5, SF = F >> 5;
@@ -607,8 +606,7 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
     const int sb = scale_byte_from_amax(m);
     const float inv = inv_scale_from_byte(sb);
     const uint64_t n0 = (uint64_t(g) * uint64_t(R) + uint64_t(r)) * uint64_t(C) + uint64_t(c0);
-    PhiloxKeys keys;
-    if constexpr (SR) keys = philox_keys(a.sr_key0, a.sr_key1);
+    const PhiloxKeys& keys = a.sr_keys;   // kernel parameters: read from the constant bank
     uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
     uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
     uint32_t w[4] = {q0.x, q0.y, q1.x, q1.y};  // 32 codes of row r, nibble k = element k
@@ -682,7 +680,7 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
 constexpr int kQ2dWarps = 8;   // warps (blocks) per CTA
 
 template <typename InT, bool RHT, bool SR, bool DEOSC>
-__global__ void __launch_bounds__(kQ2dWarps * 32, 4) quant2d_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kQ2dWarps * 32, 4) quant2d_kernel(const __grid_constant__ QuantArgs a) {
     // Per warp: the block as 32 rows x 8 chunks of 4 binary32 (chunk c of row
     // r at slot c ^ (r & 7)), and its 32 x 32 state bytes (word c of row r at
     // slot c ^ ((r >> 2) & 7)); both swizzles keep the row-of-4-rows writes
@@ -809,7 +807,7 @@ __device__ __forceinline__ void nib_swap(uint32_t (&w)[4]) {
 }
 
 template <typename InT, bool DEOSC>
-__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(QuantArgs a) {
+__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(const __grid_constant__ QuantArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, c = lane & 7;
     const int64_t R = a.rows, C = a.cols;
