@@ -227,13 +227,17 @@ mxfp4_status launch_2d(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream
     const int64_t nblocks = qa.groups * (qa.rows / 32) * (qa.cols / 32);
     constexpr int kThreads2d = mxfp4::kQ2dWarps * 32;   // warps of a CTA take neighbouring blocks of a block row
     const unsigned grid = unsigned((nblocks + mxfp4::kQ2dWarps - 1) / mxfp4::kQ2dWarps);
+    // the coalesced kernel: one CTA per tile of kCoalBlkRows x kCoalBlkCols blocks in every group
+    const int64_t tiles2 = ((qa.rows / 32 + mxfp4::kCoalBlkRows - 1) / mxfp4::kCoalBlkRows) *
+                           ((qa.cols / 32 + mxfp4::kCoalBlkCols - 1) / mxfp4::kCoalBlkCols);
+    const unsigned grid_coal = unsigned(qa.groups * tiles2);
     if constexpr (DEOSC) {
-        mxfp4::quant2d_coal_kernel<InT, true><<<grid, kThreads2d, 0, st>>>(qa);
+        mxfp4::quant2d_coal_kernel<InT, true><<<grid_coal, mxfp4::kCoalWarps * 32, 0, st>>>(qa);
     } else {
         if (rht && sr) mxfp4::quant2d_kernel<InT, true, true, false><<<grid, kThreads2d, 0, st>>>(qa);
         else if (rht) mxfp4::quant2d_kernel<InT, true, false, false><<<grid, kThreads2d, 0, st>>>(qa);
         else if (sr) mxfp4::quant2d_kernel<InT, false, true, false><<<grid, kThreads2d, 0, st>>>(qa);
-        else mxfp4::quant2d_coal_kernel<InT, false><<<grid, kThreads2d, 0, st>>>(qa);
+        else mxfp4::quant2d_coal_kernel<InT, false><<<grid_coal, mxfp4::kCoalWarps * 32, 0, st>>>(qa);
     }
     return check_launch(DEOSC ? "mxfp4_deosc_update" : "mxfp4_quantize(2d)");
 }

@@ -678,6 +678,8 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
 }
 
 constexpr int kQ2dWarps = 8;   // warps (blocks) per CTA
+constexpr int kCoalBlkRows = 1, kCoalBlkCols = 8;   // the coalesced kernel's CTA: 1 x 8 blocks
+constexpr int kCoalWarps = kCoalBlkRows * kCoalBlkCols;   // one warp per block
 
 template <typename InT, bool RHT, bool SR, bool DEOSC>
 __global__ void __launch_bounds__(kQ2dWarps * 32, 4) quant2d_kernel(const __grid_constant__ QuantArgs a) {
@@ -807,17 +809,26 @@ __device__ __forceinline__ void nib_swap(uint32_t (&w)[4]) {
 }
 
 template <typename InT, bool DEOSC>
-__global__ void __launch_bounds__(kQ2dWarps * 32) quant2d_coal_kernel(const __grid_constant__ QuantArgs a) {
+__global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __grid_constant__ QuantArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = lane >> 3, c = lane & 7;
     const int64_t R = a.rows, C = a.cols;
     const int64_t nbr = R >> 5, nbc = C >> 5;
-    const int64_t nblocks = a.groups * nbr * nbc;
-    const int64_t bid = int64_t(blockIdx.x) * kQ2dWarps + warp;
-    if (bid >= nblocks) return;
-    const int64_t g = bid / (nbr * nbc);
-    const int64_t rem = bid - g * nbr * nbc;
-    const int64_t bi = rem / nbc, bj = rem - bi * nbc;
+    // A CTA takes a tile of kCoalBlkRows x kCoalBlkCols neighbouring blocks
+    // aligned to the block grid, so the row segments it reads and writes
+    // start on tile boundaries and are not shared with another CTA (a
+    // straight run of 8 blocks along a block row that wraps at the row end
+    // left CTAs sharing partly written lines).
+    const uint32_t tiles_c = uint32_t((nbc + kCoalBlkCols - 1) / kCoalBlkCols);
+    const uint32_t tiles_r = uint32_t((nbr + kCoalBlkRows - 1) / kCoalBlkRows);
+    const uint32_t per_g = tiles_r * tiles_c;
+    const uint32_t cta = blockIdx.x;
+    const int64_t g = cta / per_g;
+    const uint32_t rem = cta - uint32_t(g) * per_g;
+    const uint32_t ti = rem / tiles_c, tj = rem - ti * tiles_c;
+    const int64_t bi = int64_t(ti) * kCoalBlkRows + warp / kCoalBlkCols;
+    const int64_t bj = int64_t(tj) * kCoalBlkCols + warp % kCoalBlkCols;
+    if (g >= a.groups || bi >= nbr || bj >= nbc) return;
     const int64_t c0 = bj * 32;
     const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
     const int64_t row0 = g * R + bi * 32;   // global row of the block's row 0
