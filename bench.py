@@ -246,12 +246,12 @@ class Layer:
 # 8-expert / 4096-token layer, whose every tensor is exactly a quarter of the
 # full one, times 4.  An entry must go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": None, "deosc_down": None,
-    "dual_x": None, "dual_h": None,
-    "dual_dy_up": None, "dual_dy_down": None,
-    "fprop_up": 4 * (97.5e6 + 333.4e6), "fprop_down": 4 * (61.3e6 + 139.1e6),
-    "dgrad_up": 4 * (122.5e6 + 153.3e6), "dgrad_down": 4 * (61.3e6 + 138.9e6),
-    "wgrad_up": 4 * (78.8e6 + 471.4e6), "wgrad_down": 4 * (52.0e6 + 205.8e6),
+    "deosc_up": 4 * (664.4e6 + 240.5e6), "deosc_down": 4 * (332.4e6 + 102.8e6),
+    "dual_x": 4 * (97.4e6 + 15.9e6), "dual_h": 4 * (97.4e6 + 14.6e6),
+    "dual_dy_up": 4 * (194.7e6 + 67.8e6), "dual_dy_down": 4 * (97.4e6 + 16.6e6),
+    "fprop_up": 4 * (97.3e6 + 333.2e6), "fprop_down": 4 * (61.3e6 + 139.5e6),
+    "dgrad_up": 4 * (122.6e6 + 153.4e6), "dgrad_down": 4 * (61.3e6 + 139.1e6),
+    "wgrad_up": 4 * (78.8e6 + 471.2e6), "wgrad_down": 4 * (52.0e6 + 205.9e6),
 }
 
 KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
@@ -393,6 +393,9 @@ def barrier(pg):
 # ---------------------------------------------------------------------------
 # CPU baseline: the oracle on a bounded sample of the same step
 # ---------------------------------------------------------------------------
+CPU_SAMPLE_ROWS = 24576   # ~10 s of oracle work on the GPU machine's host cores
+
+
 def cpu_baseline_sample(rows=256, expert=0):
     """Time the oracle (as it stands) on a bounded sample of the step: the
     first `rows` routed rows of one expert through the up-projection's three
@@ -640,9 +643,10 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, secs, threads, _ = cpu_baseline_sample(rows=256)
+        v, secs, threads, _ = cpu_baseline_sample(rows=CPU_SAMPLE_ROWS)
         cpu = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": "256 routed rows of expert 0: up-projection fprop/dgrad/wgrad binary64 GEMMs plus their "
+               "sample": "%d routed rows of expert 0: up-projection fprop/dgrad/wgrad binary64 GEMMs plus their "
+                         % CPU_SAMPLE_ROWS +
                          "quantisations (2D de-oscillation W, SR dY, RHT-16 transposed operands); %.1f s on %d "
                          "threads of %d host cores" % (secs, threads, os.cpu_count() or 0)}
     ck = clocks.summary(t0, t1)
