@@ -1,7 +1,8 @@
 """GPU parity at full size, in the launch configuration bench.py times: the
 GPT-OSS-20B-shaped MoE expert layer (32 experts, d_model 2880, W_up
-5760x2880, W_down 2880x2880, 16384 tokens top-4 with Zipf(1.1) skew) and the
-200-step de-oscillation stress on 32x5760x2880 fp32 masters.
+5760x2880, W_down 2880x2880, 16384 tokens top-4 with Zipf(1.1) skew), the
+fused bf16 + MXFP4 epilogue of its fprop and dgrad, and the 200-step
+de-oscillation stress on 32x5760x2880 fp32 masters.
 
 The oracle cannot run the whole layer, so it checks sampled outputs one by
 one: for each sampled GEMM output it quantises exactly the rows (1x32), the
@@ -14,7 +15,7 @@ import torch
 
 import oracle
 from fp4_precision_numerics_b200 import mxfp4, synth
-from tests.gpu_util import dev_bf16, dev_f32, host
+from tests.gpu_util import dev_bf16, dev_f32, host, mma_scales_to_rows
 
 pytestmark = pytest.mark.gpu
 TOL = 1e-3
@@ -142,3 +143,55 @@ def test_deosc_full_size_200_steps():
             assert int(out["scales"][g, bi, bj].item()) == int(s_ref[i, 0, 0]), (step, i)
     frozen = int((st >> 7).sum().item())
     assert frozen > 0, "near-boundary weights never froze"
+
+
+def test_fused_epilogue_full_size(layer):
+    """fprop_up and dgrad_up of the full layer with the fused epilogue: the
+    bf16 output equals the binary32 path's output rounded to bf16 and its
+    codes and scales equal the library's 1x32 quantisation of that output,
+    over every element; sampled outputs lie within the GEMM bound of the
+    oracle's binary64 product plus half a bf16 step."""
+    L = layer
+    offs_h = L["offsets"]
+    M = int(offs_h[-1])
+    offs = torch.tensor(offs_h.astype(np.int32), device="cuda")
+    x, dy_up, w_up = dev_bf16(L["x"]), dev_bf16(L["dy_up"]), dev_bf16(L["w_up"])
+    qwu = mxfp4.quantize(w_up, block="32x32", scales=False, scales_mma=True, transposed=True)
+    qx = mxfp4.quantize(x, scales=False, scales_mma=True)
+    qdu = mxfp4.quantize(dy_up, sr_seed=1, sr_offset=2, scales=False, scales_mma=True)
+    cases = (("fprop_up", mxfp4.GEMM_FPROP, qx, qwu["codes"], qwu["scales_mma"], F, D),
+             ("dgrad_up", mxfp4.GEMM_DGRAD, qdu, qwu["codes_t"], qwu["scales_mma_t"], D, F))
+    rng = np.random.default_rng(12)
+    for name, op, qa, bc, bs, N, K in cases:
+        y, q = mxfp4.grouped_gemm_fused(op, offs, qa["codes"], qa["scales_mma"], bc, bs, M, N, K)
+        y32 = mxfp4.grouped_gemm(op, offs, qa["codes"], qa["scales_mma"], bc, bs, M, N, K)
+        mxfp4.mxfp4_check_device_status()
+        assert torch.equal(y.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16)), name
+        del y32
+        ql = mxfp4.quantize(y, scales=True, scales_mma=True)
+        assert torch.equal(q["codes"], ql["codes"][0]) and torch.equal(q["scales"], ql["scales"][0]), name
+        S = N // 32   # the tensor-core layout pads the last 4-scale chunk: compare the defined bytes
+        assert np.array_equal(mma_scales_to_rows(host(q["scales_mma"]), M, S),
+                              mma_scales_to_rows(host(ql["scales_mma"][0]), M, S)), name
+        del ql
+        rows = rng.integers(0, M, size=12)
+        cols = rng.integers(0, N, size=12)
+        yh = host(y[torch.from_numpy(rows).cuda()].float())
+        for i, (m, n) in enumerate(zip(rows, cols)):
+            g = int(np.searchsorted(offs_h, m, side="right") - 1)
+            if op == mxfp4.GEMM_FPROP:
+                c, s = oracle.quantize_1d(L["x"][m:m + 1], row0=int(m))
+                A = oracle.dequant_1d(c, s)[0]
+                r0 = 32 * (n // 32)
+                cw, sw = oracle.quantize_2d(L["w_up"][g, r0:r0 + 32])
+                B = oracle.dequant_2d(cw, sw)[n - r0]
+            else:
+                c, s = oracle.quantize_1d(L["dy_up"][m:m + 1], row0=int(m), sr=True, sr_seed=1, sr_offset=2)
+                A = oracle.dequant_1d(c, s)[0]
+                c0 = 32 * (n // 32)
+                cw, sw = oracle.quantize_2d(np.ascontiguousarray(L["w_up"][g][:, c0:c0 + 32]))
+                B = oracle.dequant_2d(cw, sw)[:, n - c0]
+            ref, absref = float(A @ B), float(np.abs(A) @ np.abs(B))
+            err = abs(float(yh[i, n]) - ref)
+            assert err <= TOL * absref + 2.0 ** -8 * abs(float(yh[i, n])) + 1e-30, (name, m, n, float(yh[i, n]), ref)
+        del y, q
