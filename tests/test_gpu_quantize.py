@@ -46,6 +46,14 @@ def test_student_t_sweep_smallest_shape(sr):
     _check_1d(x, dev_bf16(x), rht_seed=1, sr_seed=1 if sr else None, sr_offset=3)
 
 
+@pytest.mark.parametrize("sr", [False, True])
+def test_student_t_sweep_middle_shape(sr):
+    """16384 x 2880, every element against the oracle."""
+    R, C = synth.QUANT_SWEEP_SHAPES[1]
+    x = synth.student_t_activations(R, C, seed=1)
+    _check_1d(x, dev_bf16(x), rht_seed=1, sr_seed=1 if sr else None, sr_offset=4)
+
+
 def test_student_t_largest_shape_sampled_rows():
     """65536 x 5760 at full size (the bench's launch shape), oracle on 48
     sampled rows (SR counters use the global row index)."""
