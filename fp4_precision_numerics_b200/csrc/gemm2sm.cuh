@@ -63,7 +63,7 @@ constexpr uint32_t kOffSFA = kOffB + kStages * kBBytes;
 constexpr uint32_t kOffSFB = kOffSFA + kStages * kSFABytes;
 constexpr uint32_t kOffEpi = kOffSFB + kStages * kSFBBytes;
 constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * kEpiBufBytes;
-constexpr uint32_t kNumBars = 4 * kStages + 2 + 2 + 1;  // full, empty, sffull, sfready, tfull, tempty, drain
+constexpr uint32_t kNumBars = 3 * kStages + 2 + 2 + 1;  // full, empty, sffull, tfull, tempty, drain
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffGroups = kOffMisc + 64;
 constexpr uint32_t kOffPrefix = kOffGroups + (kMaxGroups + 1) * 4;
@@ -137,13 +137,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* full = bars;                        // leader: A/B of both CTAs landed (2 arrivals + bytes)
+    // full (leader): the stage is ready for the pair's MMAs -- A/B of both
+    // CTAs landed (2 producer arrivals + bytes) and both CTAs' scales are in
+    // tensor memory (8 loader-warp arrivals); one wait per K-step
+    uint64_t* full = bars;
     uint64_t* empty = bars + kStages;             // both: the pair's MMAs released the stage
     uint64_t* sffull = bars + 2 * kStages;        // both: this CTA's scale chunks landed
-    uint64_t* sfready = bars + 3 * kStages;       // leader: both CTAs' scales are in TMEM (8 warps)
-    uint64_t* tfull = bars + 4 * kStages;         // both: accumulator ready
-    uint64_t* tempty = bars + 4 * kStages + 2;    // leader: both CTAs drained the accumulator (8 warps)
-    uint64_t* drain = bars + 4 * kStages + 4;     // both: all of the pair's MMAs completed
+    uint64_t* tfull = bars + 3 * kStages;         // both: accumulator ready
+    uint64_t* tempty = bars + 3 * kStages + 2;    // leader: both CTAs drained the accumulator (8 warps)
+    uint64_t* drain = bars + 3 * kStages + 4;     // both: all of the pair's MMAs completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
     volatile int* offsets_ok = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
@@ -158,10 +160,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = threadIdx.x; i <= a.num_groups; i += blockDim.x) s_off[i] = __ldg(a.offsets + i);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 2);
+            mbar_init(&full[s], 2 + 8);
             mbar_init(&empty[s], 1);
             mbar_init(&sffull[s], 1);
-            mbar_init(&sfready[s], 8);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
@@ -303,8 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t d_tmem = tmem_base + acc * kAccCols;
                     bool first = true;
                     for (int64_t k = un.kbeg; k < un.kend; k += BK) {
-                        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, a.status, kRoleMma) ||
-                            !mbar_wait_bounded(&sfready[stage], phase, abort_flag, a.status, kRoleMma)) {
+                        if (!mbar_wait_bounded(&full[stage], phase, abort_flag, a.status, kRoleMma)) {
                             ok = false;
                             break;
                         }
@@ -379,7 +379,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&sfready[stage]), 0));
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&full[stage]), 0));
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1u;
