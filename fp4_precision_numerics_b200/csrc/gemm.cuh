@@ -82,6 +82,11 @@ struct Args {
     int m_tiles, n_tiles;     // mode 0: over all rows of A; mode 1: per group
     int64_t total_tiles;
     uint32_t* status;
+    // CTA-pair kernel: a K-step loads A and B with one box each through views
+    // [chunk][row][256 bytes] of the codes (chunk stride 128 B); k_chunks is
+    // the number of chunk positions whose 256 bytes lie inside a row, 0 if
+    // the views are not used
+    int32_t k_chunks;
     // fused epilogue (CTA-pair kernel, mode 0 only): bf16 output and its MXFP4
     // quantisation in 1x32 blocks along N, in place of the binary32 output
     // (bf16 [M][ldy] and codes [M][N/2] leave through tensor maps)

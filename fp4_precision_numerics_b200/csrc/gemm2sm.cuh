@@ -133,6 +133,7 @@ template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
+                            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                             const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,6 +176,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmD);
         if constexpr (FUSED) prefetch_tensormap(&tmQ);
+        if (a.k_chunks > 0) {
+            prefetch_tensormap(&tmA2);
+            prefetch_tensormap(&tmB2);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -246,13 +251,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     uint8_t* sA = smem + kOffA + stage * kABytes;
                     uint8_t* sB = smem + kOffB + stage * kBBytes;
                     const int32_t brow = int32_t(un.n0 + BNH * int64_t(rank));
-                    for (int j = 0; j < nsub; ++j) {
-                        const int32_t xk = int32_t((k + 256 * j) >> 1);
-                        tma_load_2d_pair(sA + j * kABox, &tmA, full_c, xk, int32_t(mt * BM));
+                    // the K-step's 256 bytes per row start at byte k/2: chunk kc,
+                    // offset xo (0 or 64) inside it
+                    const int32_t kc = int32_t(k >> 8), xo = int32_t((k >> 1) & 127);
+                    if (nsub == 2 && kc + 2 <= a.k_chunks) {
+                        // both halves in one box each for A and B
+                        tma_load_3d_pair(sA, &tmA2, full_c, xo, int32_t(mt * BM), kc);
                         if (a.mode == 0)
-                            tma_load_3d_pair(sB + j * kBBox, &tmB, full_c, xk, brow, un.g);
+                            tma_load_4d_pair(sB, &tmB2, full_c, xo, brow, kc, un.g);
                         else
-                            tma_load_2d_pair(sB + j * kBBox, &tmB, full_c, xk, brow);
+                            tma_load_3d_pair(sB, &tmB2, full_c, xo, brow, kc);
+                    } else {
+                        for (int j = 0; j < nsub; ++j) {
+                            const int32_t xk = int32_t((k + 256 * j) >> 1);
+                            tma_load_2d_pair(sA + j * kABox, &tmA, full_c, xk, int32_t(mt * BM));
+                            if (a.mode == 0)
+                                tma_load_3d_pair(sB + j * kBBox, &tmB, full_c, xk, brow, un.g);
+                            else
+                                tma_load_2d_pair(sB + j * kBBox, &tmB, full_c, xk, brow);
+                        }
                     }
                     pend[stage] = true;
                     pend_phase[stage] = phase;

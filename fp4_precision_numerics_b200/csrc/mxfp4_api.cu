@@ -275,8 +275,9 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base
               const uint64_t* strides_bytes, const uint32_t* box) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t d[3], s[2];
-    cuuint32_t b[3], e[3] = {1, 1, 1};
+    if (rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], e[5] = {1, 1, 1, 1, 1};
     for (int i = 0; i < rank; ++i) {
         d[i] = dims[i];
         b[i] = box[i];
@@ -291,8 +292,9 @@ bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void
                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t d[3], s[2];
-    cuuint32_t b[3], e[3] = {1, 1, 1};
+    if (rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], e[5] = {1, 1, 1, 1, 1};
     for (int i = 0; i < rank; ++i) {
         d[i] = dims[i];
         b[i] = box[i];
@@ -421,7 +423,37 @@ mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offs
     if (pair) {
         namespace g2 = mxfp4::gemm2;
         if (!f) tmQ = tmA;   // unused by the binary32 epilogue
-        void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const Args) =
+        // two-chunk views: each row of K/2 bytes seen as [chunk][row][256
+        // bytes] with a chunk stride of 128 B, so one 128-byte-wide box of two
+        // chunks carries both 256-element halves of a K-step, starting at byte
+        // offset 0 or 64 of its first chunk (wgrad's expert ranges start on
+        // 128-token boundaries).  Only chunk positions whose 256 bytes lie
+        // inside the row are in the view.
+        CUtensorMap tmA2 = tmA, tmB2 = tmB;
+        const uint64_t nch = kb >= 256 ? (kb - 256) / 128 + 1 : 0;
+        a.k_chunks = int32_t(nch >= 2 ? nch : 0);
+        if (a.k_chunks > 0) {
+            const uint64_t dimsA[3] = {256, uint64_t(M), nch};
+            const uint64_t strA[2] = {kb, 128};
+            const uint32_t boxA[3] = {128, BM, 2};
+            if (!make_map(&tmA2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, A.codes, dimsA, strA, boxA))
+                return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for A (whole chunks) failed");
+            if (a.mode == 0) {
+                const uint64_t dimsB[4] = {256, uint64_t(N), nch, uint64_t(num_groups)};
+                const uint64_t strB[3] = {kb, 128, kb * uint64_t(N)};
+                const uint32_t boxB[4] = {128, b_rows, 2, 1};
+                if (!make_map(&tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, B.codes, dimsB, strB, boxB))
+                    return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B (whole chunks) failed");
+            } else {
+                const uint64_t dimsB[3] = {256, uint64_t(N), nch};
+                const uint64_t strB[2] = {kb, 128};
+                const uint32_t boxB[3] = {128, b_rows, 2};
+                if (!make_map(&tmB2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, B.codes, dimsB, strB, boxB))
+                    return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B (whole chunks) failed");
+            }
+        }
+        void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                     const CUtensorMap, const Args) =
             f ? g2::grouped_gemm_2sm_kernel<true> : g2::grouped_gemm_2sm_kernel<false>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g2::kSmemBytes) != cudaSuccess)
             return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
@@ -432,7 +464,8 @@ mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offs
         if (units == 0) return ok();
         const int64_t clusters = pair_clusters();
         const unsigned grid = 2u * unsigned(units < clusters ? units : clusters);
-        kern<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, tmQ, a);
+        kern<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, tmQ, tmA2, tmB2,
+                                                                                       a);
         return check_launch("mxfp4_grouped_gemm");
     }
     if (f) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: needs the CTA-pair kernel");
