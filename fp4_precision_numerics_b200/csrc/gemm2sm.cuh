@@ -236,16 +236,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t nca = uint32_t(imin64(kChunks, a.nchunk_a - chunk));
                     const uint32_t ncb = uint32_t(imin64(kChunks, a.nchunk_b - chunk));
                     const int nsub = un.kend - k > 256 ? 2 : 1;   // boxes of 256 elements this K-step needs
-                    // scales first: they are small, and the loader warps move them
-                    // to tensor memory while the operand tiles are still in flight
-                    mbar_arrive_expect_tx(&sffull[stage], nca * 512u + ncb * 512u * (has_rb1 ? 2u : 1u));
-                    bulk_load(smem + kOffSFA + stage * kSFABytes, a.sfa + (mt * a.nchunk_a + chunk) * 512, nca * 512u,
-                              &sffull[stage]);
-                    bulk_load(smem + kOffSFB + stage * kSFBBytes, sfb_g + (rbb * a.nchunk_b + chunk) * 512,
-                              ncb * 512u, &sffull[stage]);
-                    if (has_rb1)
-                        bulk_load(smem + kOffSFB + stage * kSFBBytes + kChunks * 512,
-                                  sfb_g + ((rbb + 1) * a.nchunk_b + chunk) * 512, ncb * 512u, &sffull[stage]);
                     const uint32_t full_c = mapa_shared(smem_u32(&full[stage]), 0);
                     mbar_arrive_expect_tx_cluster(full_c, uint32_t(nsub) * (kABox + kBBox));
                     uint8_t* sA = smem + kOffA + stage * kABytes;
@@ -271,6 +261,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 tma_load_2d_pair(sB + j * kBBox, &tmB, full_c, xk, brow);
                         }
                     }
+                    // then the scales: small, they reach tensor memory (bulk copy,
+                    // loader warps) well before the operand tiles land, so the
+                    // operand copies go first
+                    mbar_arrive_expect_tx(&sffull[stage], nca * 512u + ncb * 512u * (has_rb1 ? 2u : 1u));
+                    bulk_load(smem + kOffSFA + stage * kSFABytes, a.sfa + (mt * a.nchunk_a + chunk) * 512, nca * 512u,
+                              &sffull[stage]);
+                    bulk_load(smem + kOffSFB + stage * kSFBBytes, sfb_g + (rbb * a.nchunk_b + chunk) * 512,
+                              ncb * 512u, &sffull[stage]);
+                    if (has_rb1)
+                        bulk_load(smem + kOffSFB + stage * kSFBBytes + kChunks * 512,
+                                  sfb_g + ((rbb + 1) * a.nchunk_b + chunk) * 512, ncb * 512u, &sffull[stage]);
                     pend[stage] = true;
                     pend_phase[stage] = phase;
                     if (++stage == kStages) {
