@@ -40,6 +40,8 @@ WORKLOAD = ("GPT-OSS-20B-shaped MoE expert layer, full MXFP4 training step (fpro
             "W_down 2880x2880, 16384 tokens top-4 Zipf(1.1)")
 E, D, F = 32, 2880, 5760
 NOMINAL_FP4_OVER_BF16 = 4.0          # dense FP4 / dense BF16 tensor rate, B200 datasheet (9 / 2.25 PFLOP/s)
+NOMINAL_HBM_GBS = 8000.0             # B200 HBM3e, datasheet
+NOMINAL_FP4_TFLOPS = 9000.0          # B200 dense FP4, datasheet
 
 
 def load_peaks():
@@ -539,12 +541,14 @@ def main():
                 "peak_source": "%s sustained bf16 x %.0f (nominal FP4:BF16 dense ratio)" % (peaks["source"],
                                                                                           NOMINAL_FP4_OVER_BF16),
                 "kernel": dominant, "traffic": dom_traffic,
-                "hbm_frac": layer.gemm_out_bytes(dominant) / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                "hbm_frac": layer.gemm_out_bytes(dominant) / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                "peak_nominal": NOMINAL_FP4_TFLOPS, "frac_nominal": achieved / NOMINAL_FP4_TFLOPS}
     else:
         achieved = layer.quant_bytes[dominant] / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                "kernel": dominant, "traffic": dom_traffic}
+                "kernel": dominant, "traffic": dom_traffic,
+                "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": achieved / NOMINAL_HBM_GBS}
     components = {}
     for k in KERNELS:
         t = per_kernel[k]
@@ -660,6 +664,8 @@ def main():
                    "experts": E, "parallelism": "replica per GPU" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (working set ~14 GB per step)"},
         "quantise_gbs": quant_gbs, "quantise_frac_hbm": quant_gbs / peaks["hbm_gbs"],
+        "quantise_frac_hbm_nominal": quant_gbs / NOMINAL_HBM_GBS,
+        "gemm_frac_fp4_nominal": step_flops / (gemm_ms / 1e3) / 1e12 / NOMINAL_FP4_TFLOPS,
         "gemm_tflops": step_flops / (gemm_ms / 1e3) / 1e12, "gemm_frac_fp4": step_flops / (gemm_ms / 1e3) / 1e12 / fp4_peak,
         "roofline": roof, "components": components,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d_bytes),
