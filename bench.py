@@ -432,6 +432,78 @@ def cpu_baseline_sample(rows=256, expert=0):
     return flops / secs / 1e12, secs, oracle.num_threads(), flops
 
 
+def oracle_timing():
+    """A fuller timing report of the oracle (part of the CPU-baseline leg):
+    the 1x32 quantisation of the three sweep shapes at full size with every
+    host thread, the smallest shape on one thread, the plain binary64 GEMM
+    loop on the single layer and on the smallest expert of the MoE layer,
+    and the numpy binary64 GEMMs of the layer's fprop (up and down)."""
+    import subprocess
+
+    import numpy as np
+
+    import oracle
+    from fp4_precision_numerics_b200 import synth
+    oracle.lib()
+    rep = {"threads": oracle.num_threads(), "host_cores": os.cpu_count()}
+    qs = []
+    for (R, C) in synth.QUANT_SWEEP_SHAPES:
+        x = synth.student_t_activations(R, C, seed=0)
+        for sr in (False, True):
+            t0 = time.perf_counter()
+            oracle.quantize_1d(x, rht_d=16, rht_seed=1, sr=sr, sr_seed=1)
+            dt = time.perf_counter() - t0
+            qs.append({"shape": [R, C], "sr": sr, "s": round(dt, 3), "gbs": round(R * C * 2.53125 / dt / 1e9, 3)})
+        del x
+    rep["quantise_all_threads"] = qs
+    R, C = synth.QUANT_SWEEP_SHAPES[0]
+    code = ("import time, sys; sys.path.insert(0, %r); import oracle; from fp4_precision_numerics_b200 import synth; "
+            "x = synth.student_t_activations(%d, %d, seed=0); oracle.lib(); t0 = time.perf_counter(); "
+            "oracle.quantize_1d(x, rht_d=16, rht_seed=1, sr=True, sr_seed=1); print(time.perf_counter() - t0)"
+            % (ROOT, R, C))
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, check=True)
+    dt1 = float(out.stdout.strip().splitlines()[-1])
+    rep["quantise_one_thread"] = {"shape": [R, C], "sr": True, "s": round(dt1, 3),
+                                  "gbs": round(R * C * 2.53125 / dt1 / 1e9, 3)}
+    x, w = synth.single_layer(seed=0)
+    A, B = synth.bf16_to_f32(x).astype(np.float64), synth.bf16_to_f32(w).astype(np.float64)
+    t0 = time.perf_counter()
+    oracle.gemm_f64_loop(A, B)
+    dt = time.perf_counter() - t0
+    rep["gemm_loop_single_layer"] = {"flop": 2 * 256 ** 3, "s": round(dt, 4), "gflops": round(2 * 256 ** 3 / dt / 1e9, 3)}
+    L = synth.moe_layer(with_grads=False)
+    off, counts = L["offsets"], L["counts"]
+    e = int(np.argmin(counts))
+    lo, hi = int(off[e]), int(off[e + 1])
+    cx, sx = oracle.quantize_1d(L["x"][lo:hi])
+    Xq = oracle.dequant_1d(cx, sx)
+    cw, sw = oracle.quantize_2d(L["w_up"][e])
+    Wq = oracle.dequant_2d(cw, sw)
+    fl = 2.0 * (hi - lo) * Wq.shape[0] * Wq.shape[1]
+    t0 = time.perf_counter()
+    oracle.gemm_f64_loop(Xq, Wq)
+    dt = time.perf_counter() - t0
+    rep["gemm_loop_smallest_expert"] = {"expert": e, "rows": hi - lo, "routed_rows": int(counts[e]), "flop": fl,
+                                        "s": round(dt, 2), "gflops": round(fl / dt / 1e9, 3)}
+    cx, sx = oracle.quantize_1d(L["x"])
+    Xq = oracle.dequant_1d(cx, sx)
+    ch, sh = oracle.quantize_1d(L["h"])
+    Hq = oracle.dequant_1d(ch, sh)
+    E = len(counts)
+    Wu = np.stack([oracle.dequant_2d(*oracle.quantize_2d(L["w_up"][g])) for g in range(E)])
+    Wd = np.stack([oracle.dequant_2d(*oracle.quantize_2d(L["w_down"][g])) for g in range(E)])
+    fl = 2.0 * float(counts.sum()) * (Wu.shape[1] * Wu.shape[2] + Wd.shape[1] * Wd.shape[2])
+    t0 = time.perf_counter()
+    oracle.grouped_gemm_f64(Xq, Wu, off)
+    oracle.grouped_gemm_f64(Hq, Wd, off)
+    dt = time.perf_counter() - t0
+    rep["numpy_fprop_up_down"] = {"flop": fl, "s": round(dt, 2), "tflops": round(fl / dt / 1e12, 4),
+                                  "note": "numpy binary64 matmul on dequantised operands; the training step is 3x "
+                                          "this work (dgrad and wgrad have the same FLOPs)"}
+    return rep
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -470,6 +542,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-timing", action="store_true",
+                    help="print a fuller timing report of the CPU oracle (host only) and exit")
     ap.add_argument("--fused-steps", type=int, default=10,
                     help="steps of the fused-epilogue variant timed after the main region (0: skip)")
     ap.add_argument("--experts", type=int, default=32,
@@ -480,6 +554,9 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.oracle_timing:
+        print(json.dumps({"oracle_timing": oracle_timing()}))
+        return 0
 
     import torch
     rank, world, local, pg = dist_setup(args.gpus)
