@@ -504,6 +504,48 @@ def oracle_timing():
     return rep
 
 
+def quant_sweep(iters=20, warmup=3):
+    """GPU timing of the 1x32 quantiser alone on the quantise-sweep shapes
+    (bf16 Gaussian draws on the device -- the kernels' time does not depend
+    on the values --, RHT-16, nearest and stochastic rounding):
+    median of `iters` CUDA-event timings after `warmup`, with L2 flushed
+    (a 256 MB write) before every timed launch.  Bytes per element: 2 in,
+    1/2 + 1/32 out."""
+    import numpy as np
+    import torch
+
+    from fp4_precision_numerics_b200 import mxfp4, synth
+    peaks = load_peaks()
+    dev = torch.device("cuda", 0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for (R, C) in synth.QUANT_SWEEP_SHAPES:
+        g = torch.Generator(device=dev)
+        g.manual_seed(R + C)
+        x = torch.randn((R, C), generator=g, device=dev).to(torch.bfloat16)
+        out = dict(codes=torch.empty((1, R, C // 2), dtype=torch.uint8, device=dev),
+                   scales=torch.empty((1, R, C // 32), dtype=torch.uint8, device=dev))
+        for sr in (False, True):
+            ts = []
+            for i in range(warmup + iters):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                mxfp4.quantize(x, rht_seed=1, sr_seed=1 if sr else None, sr_offset=i, scales=True, out=out)
+                e1.record()
+                torch.cuda.synchronize()
+                if i >= warmup:
+                    ts.append(e0.elapsed_time(e1))
+            ms = float(np.median(ts))
+            gbs = R * C * (2 + 0.5 + 1.0 / 32) / (ms / 1e3) / 1e9
+            rows.append({"shape": [R, C], "sr": sr, "ms": round(ms, 4), "gbs": round(gbs, 1),
+                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "frac_hbm_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
+        del x, out
+    mxfp4.mxfp4_check_device_status()
+    return {"quant_sweep": rows, "l2": "flushed (256 MB write) before every timed launch", "iters": iters,
+            "warmup": warmup, "peak_source": peaks["source"] + " copy bandwidth"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -542,6 +584,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quant-sweep", action="store_true",
+                    help="time the 1x32 quantiser alone on the quantise-sweep shapes (L2 flushed) and exit")
     ap.add_argument("--oracle-timing", action="store_true",
                     help="print a fuller timing report of the CPU oracle (host only) and exit")
     ap.add_argument("--fused-steps", type=int, default=10,
@@ -556,6 +600,9 @@ def main():
         return run_reference(args)
     if args.oracle_timing:
         print(json.dumps({"oracle_timing": oracle_timing()}))
+        return 0
+    if args.quant_sweep:
+        print(json.dumps(quant_sweep()))
         return 0
 
     import torch

@@ -137,6 +137,9 @@ unsigned grid_for(int64_t work, int threads) {
 // --- quantisation launchers --------------------------------------------------
 template <typename InT>
 mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStream_t st) {
+    // the kernel indexes the rows of all groups in 32 bits
+    if (qa.groups * qa.rows >= (int64_t(1) << 31))
+        return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize: groups * rows must be < 2^31");
     const int64_t work = qa.groups * qa.rows * (qa.cols / 32);
     const unsigned grid = grid_for(work, 256);
     if (rht && sr) mxfp4::quant1d_rows_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);

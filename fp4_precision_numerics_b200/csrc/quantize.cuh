@@ -29,6 +29,14 @@ __host__ __device__ __forceinline__ int64_t mma_scale_bytes(int64_t R, int64_t S
     return ((R + 127) / 128) * ((S + 3) / 4) * 512;
 }
 
+// Byte offset of scale (r, s) in the tensor-core layout of one group whose
+// scale matrix has `nchunk` 4-scale chunks per row (32-bit form of
+// mma_scale_offset, for groups below 4 GB of scales).
+__device__ __forceinline__ uint32_t mma_off32(uint32_t r, uint32_t s, uint32_t nchunk) {
+    return ((r >> 7) * nchunk + (s >> 2)) * 512u + (r & 31u) * 16u + ((r >> 3) & 12u) + (s & 3u);
+}
+
+
 struct QuantArgs {
     const void* in;
     int64_t groups, rows, cols, ld;   // input geometry (per group: rows x cols, row stride ld)
@@ -181,35 +189,50 @@ __device__ __forceinline__ uint2 quant16(const float (&x)[16], float inv_scale, 
 // ---------------------------------------------------------------------------
 template <typename InT, bool RHT, bool SR>
 __global__ void __launch_bounds__(256) quant1d_rows_kernel(const __grid_constant__ QuantArgs a) {
-    const int64_t C = a.cols;
-    const int64_t S = C >> 5;
-    const int64_t total = a.groups * a.rows * S;
-    const int64_t mma_group_bytes = mma_scale_bytes(a.rows, S);
+    // block i = (row, s) of the [groups * rows, cols / 32] block grid, and the
+    // row's group g and row r inside it, are advanced by the grid stride with
+    // adds and one conditional wrap each (no division in the loop; the host
+    // keeps groups * rows below 2^31)
+    const uint32_t C = uint32_t(a.cols), S = C >> 5, R = uint32_t(a.rows);
+    const uint64_t total = uint64_t(a.groups) * R * S;
+    const uint32_t stride = gridDim.x * blockDim.x;
+    const uint32_t i0 = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i0 >= total) return;
+    uint32_t row = i0 / S, s = i0 - row * S;
+    uint32_t g = row / R, r = row - g * R;
+    const uint32_t drow = stride / S, ds = stride - drow * S;
+    const uint32_t dg = drow / R, dr = drow - dg * R;
+    const uint32_t nchunk = (S + 3) >> 2;
+    const uint64_t mma_group_bytes = uint64_t((R + 127) >> 7) * nchunk * 512u;
     const InT* in = static_cast<const InT*>(a.in);
-    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     const PhiloxKeys& keys = a.sr_keys;   // kernel parameters: read from the constant bank
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
-        const int64_t row = i / S;
-        const int64_t s = i - row * S;
-        const int64_t col0 = s << 5;
+    for (uint64_t i = i0; i < total; i += stride) {
+        const uint32_t col0 = s << 5;
         float x0[16], x1[16];
-        Loader<InT>::load16(in + row * a.ld + col0, x0);
-        Loader<InT>::load16(in + row * a.ld + col0 + 16, x1);
+        const InT* src = in + uint64_t(row) * uint64_t(a.ld) + col0;
+        Loader<InT>::load16(src, x0);
+        Loader<InT>::load16(src + 16, x1);
         if constexpr (RHT) {
             rht16(x0, a.rht_signs);
             rht16(x1, a.rht_signs);
         }
         const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
         const float inv = inv_scale_from_byte(sb);
-        const uint64_t n0 = uint64_t(row) * uint64_t(C) + uint64_t(col0);
+        const uint64_t n0 = uint64_t(row) * C + col0;
         const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.sr_offset);
         const uint2 q1 = quant16<SR>(x1, inv, n0 + 16, keys, a.sr_offset);
-        *reinterpret_cast<uint4*>(a.codes + row * (C >> 1) + (col0 >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+        *reinterpret_cast<uint4*>(a.codes + uint64_t(row) * (C >> 1) + (col0 >> 1)) = make_uint4(q0.x, q0.y, q1.x, q1.y);
         if (a.scales) a.scales[i] = uint8_t(sb);
-        if (a.scales_mma) {
-            const int64_t g = row / a.rows, r = row - g * a.rows;
-            a.scales_mma[g * mma_group_bytes + mma_scale_offset(r, s, S)] = uint8_t(sb);
-        }
+        if (a.scales_mma) a.scales_mma[g * mma_group_bytes + mma_off32(r, s, nchunk)] = uint8_t(sb);
+        // advance by the grid stride
+        s += ds;
+        const uint32_t cs = s >= S ? 1u : 0u;
+        s -= cs * S;
+        row += drow + cs;
+        r += dr + cs;
+        const uint32_t cr = r >= R ? 1u : 0u;
+        r -= cr * R;
+        g += dg + cr;
     }
 }
 
@@ -271,13 +294,6 @@ struct TileWalk {
         g += sg + c2;
     }
 };
-
-// Byte offset of scale (r, s) in the tensor-core layout of one group whose
-// scale matrix has `nchunk` 4-scale chunks per row (32-bit form of
-// mma_scale_offset, for groups below 4 GB of scales).
-__device__ __forceinline__ uint32_t mma_off32(uint32_t r, uint32_t s, uint32_t nchunk) {
-    return ((r >> 7) * nchunk + (s >> 2)) * 512u + (r & 31u) * 16u + ((r >> 3) & 12u) + (s & 3u);
-}
 
 // Dual mode (DUAL): every tile is also quantised in 1x32 blocks along the
 // features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
