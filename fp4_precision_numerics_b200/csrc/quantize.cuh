@@ -213,8 +213,14 @@ __global__ void __launch_bounds__(256) quant1d_rows_kernel(const __grid_constant
         Loader<InT>::load16(src, x0);
         Loader<InT>::load16(src + 16, x1);
         if constexpr (RHT) {
-            rht16(x0, a.rht_signs);
-            rht16(x1, a.rht_signs);
+            // the block's two 16-element chunks take the same butterflies:
+            // run them two-wide as (chunk 0 element i, chunk 1 element i)
+            uint64_t p[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) p[k] = f2_pack(x0[k], x1[k]);
+            rht16x2(p, a.rht_mul2);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) f2_unpack(p[k], x0[k], x1[k]);
         }
         const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
         const float inv = inv_scale_from_byte(sb);
