@@ -629,6 +629,7 @@ mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, i
     qa.r_scales = row_out->scales;
     qa.r_scales_mma = row_out->scales_mma;
     qa.r_rht_signs = rp->rht_d == 16 ? rht_sign_mask(rp->rht_seed) : 0u;
+    fill_rht_mul2(qa.r_rht_mul2, qa.r_rht_signs);
     qa.r_sr_offset = rp->sr_offset;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     return in_dtype == MXFP4_DTYPE_BF16 ? launch_dual<uint16_t>(qa, cp->rht_d == 16, rp->rht_d == 16, sr, st)

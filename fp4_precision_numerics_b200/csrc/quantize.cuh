@@ -58,6 +58,7 @@ struct QuantArgs {
     uint8_t* r_scales;
     uint8_t* r_scales_mma;
     uint32_t r_rht_signs;
+    uint64_t r_rht_mul2[16];          // packed (s_i / 4, s_i / 4) of the row-direction RHT
     uint32_t r_sr_offset;
 };
 
@@ -139,6 +140,17 @@ __device__ __forceinline__ void rht16x2(uint64_t (&p)[16], const uint64_t (&mul2
     }
 }
 
+// rht16 of a 32-element block's two 16-element chunks, run two-wide as
+// packed pairs (x0[i], x1[i]); `mul2` as for rht16x2.
+__device__ __forceinline__ void rht16_pair(float (&x0)[16], float (&x1)[16], const uint64_t (&mul2)[16]) {
+    uint64_t p[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) p[k] = f2_pack(x0[k], x1[k]);
+    rht16x2(p, mul2);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) f2_unpack(p[k], x0[k], x1[k]);
+}
+
 __device__ __forceinline__ float amax16(const float (&x)[16]) {
     float m = fmax3_abs(x[0], x[1], x[2]);
 #pragma unroll
@@ -213,14 +225,8 @@ __global__ void __launch_bounds__(256) quant1d_rows_kernel(const __grid_constant
         Loader<InT>::load16(src, x0);
         Loader<InT>::load16(src + 16, x1);
         if constexpr (RHT) {
-            // the block's two 16-element chunks take the same butterflies:
-            // run them two-wide as (chunk 0 element i, chunk 1 element i)
-            uint64_t p[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) p[k] = f2_pack(x0[k], x1[k]);
-            rht16x2(p, a.rht_mul2);
-#pragma unroll
-            for (int k = 0; k < 16; ++k) f2_unpack(p[k], x0[k], x1[k]);
+            // the block's two 16-element chunks take the same butterflies
+            rht16_pair(x0, x1, a.rht_mul2);
         }
         const int sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
         const float inv = inv_scale_from_byte(sb);
@@ -521,10 +527,7 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                     }
                     float (&x0)[16] = *reinterpret_cast<float(*)[16]>(&x[0]);
                     float (&x1)[16] = *reinterpret_cast<float(*)[16]>(&x[16]);
-                    if constexpr (RHT_R) {
-                        rht16(x0, a.r_rht_signs);
-                        rht16(x1, a.r_rht_signs);
-                    }
+                    if constexpr (RHT_R) rht16_pair(x0, x1, a.r_rht_mul2);
                     sb = scale_byte_from_amax(fmaxf(amax16(x0), amax16(x1)));
                     const float inv = inv_scale_from_byte(sb);
                     const uint2 q0 = quant16<SR>(x0, inv, n0, keys, a.r_sr_offset);
@@ -618,10 +621,7 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
     const int64_t nbr = R >> 5, nbc = C >> 5;
     const int64_t r = bi * 32 + lane;
     const int64_t c0 = bj * 32;
-    if constexpr (RHT) {
-        rht16(x0, a.rht_signs);
-        rht16(x1, a.rht_signs);
-    }
+    if constexpr (RHT) rht16_pair(x0, x1, a.rht_mul2);
     float m = fmaxf(amax16(x0), amax16(x1));
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
