@@ -87,6 +87,9 @@ struct Args {
     // the number of chunk positions whose 256 bytes lie inside a row, 0 if
     // the views are not used
     int32_t k_chunks;
+    // CTA-pair kernel, binary32 epilogue: store two 32-column chunks per TMA
+    // box through a view [column block][row][32 floats] of D (N % 32 == 0)
+    int32_t d_pairs;
     // fused epilogue (CTA-pair kernel, mode 0 only): bf16 output and its MXFP4
     // quantisation in 1x32 blocks along N, in place of the binary32 output
     // (bf16 [M][ldy] and codes [M][N/2] leave through tensor maps)

@@ -134,7 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmD, const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                            const Args a) {
+                            const __grid_constant__ CUtensorMap tmD2, const Args a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -499,6 +499,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         if (a.qscales_mma) a.qscales_mma[mma_scale_offset(grow, s, SN)] = uint8_t(sbyte);
                     }
                     buf ^= 1u;
+                    continue;
+                }
+                if (a.d_pairs) {
+                    // two 32-column chunks per store: chunk c into buffer c & 1,
+                    // one 8 KB box [2][32 rows][32 floats] after the odd chunk
+                    if ((c & 1) == 0 && lane == 0) bulk_wait_read<0>();
+                    __syncwarp();
+                    uint8_t* sb = stg + (c & 1) * kEpiBufBytes;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int pos = j ^ (lane & 7);
+                        *reinterpret_cast<uint4*>(sb + lane * 128 + pos * 16) =
+                            make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                    }
+                    if (c & 1) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            const int64_t col = un.n0 + 32 * (c - 1);
+                            if (col < a.N && row < a.M) {
+                                if (a.mode == 0)
+                                    tma_store_3d(&tmD2, stg, 0, int32_t(row), int32_t(col >> 5));
+                                else
+                                    tma_store_4d(&tmD2, stg, 0, int32_t(row), int32_t(col >> 5), un.g);
+                            }
+                            bulk_commit();
+                        }
+                    }
                     continue;
                 }
                 if (lane == 0) bulk_wait_read<1>();

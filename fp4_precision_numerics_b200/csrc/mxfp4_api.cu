@@ -62,6 +62,9 @@ int64_t resident_ctas(K kern, int threads, size_t smem) {
     return int64_t(num_sms()) * per_sm;
 }
 
+// The pair GEMM's binary32 epilogue stores two 32-column chunks per TMA box.
+constexpr bool kEpiPairStores = true;
+
 // Clusters of two CTAs of the pair GEMM that can be resident at once (one
 // CTA per SM; an SM left without a partner in its GPC stays idle).
 int pair_clusters() {
@@ -455,8 +458,28 @@ mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offs
                     return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for B (whole chunks) failed");
             }
         }
+        // binary32 output seen as [column block][row][32 floats] (column-block
+        // stride 128 B), so one 32 x 32 x 2 box stores two chunks
+        CUtensorMap tmD2 = tmD;
+        a.d_pairs = 0;
+        if (!f && N % 32 == 0 && kEpiPairStores) {
+            bool okm;
+            if (a.mode == 0) {
+                const uint64_t dd[3] = {32, uint64_t(M), uint64_t(N / 32)};
+                const uint64_t ds[2] = {uint64_t(ldo) * 4, 128};
+                const uint32_t db[3] = {32, 32, 2};
+                okm = make_map(&tmD2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dd, ds, db);
+            } else {
+                const uint64_t dd[4] = {32, uint64_t(M), uint64_t(N / 32), uint64_t(num_groups)};
+                const uint64_t ds[3] = {uint64_t(ldo) * 4, 128, uint64_t(ldo) * 4 * uint64_t(M)};
+                const uint32_t db[4] = {32, 32, 2, 1};
+                okm = make_map(&tmD2, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out, dd, ds, db);
+            }
+            if (!okm) return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: tensor map for D (chunk pairs) failed");
+            a.d_pairs = 1;
+        }
         void (*kern)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap, const CUtensorMap,
-                     const CUtensorMap, const Args) =
+                     const CUtensorMap, const CUtensorMap, const Args) =
             f ? g2::grouped_gemm_2sm_kernel<true> : g2::grouped_gemm_2sm_kernel<false>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, g2::kSmemBytes) != cudaSuccess)
             return fail(MXFP4_ERR_CUDA, "mxfp4_grouped_gemm: cannot raise the shared-memory limit");
@@ -468,7 +491,7 @@ mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offs
         const int64_t clusters = pair_clusters();
         const unsigned grid = 2u * unsigned(units < clusters ? units : clusters);
         kern<<<grid, g2::kThreads, g2::kSmemBytes, static_cast<cudaStream_t>(stream)>>>(tmA, tmB, tmD, tmQ, tmA2, tmB2,
-                                                                                       a);
+                                                                                       tmD2, a);
         return check_launch("mxfp4_grouped_gemm");
     }
     if (f) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: needs the CTA-pair kernel");
