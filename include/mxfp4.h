@@ -127,8 +127,9 @@ MXFP4_API size_t mxfp4_mma_scale_bytes(int64_t rows, int64_t nscales);
  *  layout  : 1D along the last dim -> output [rows, cols]; 1D along rows ->
  *            output [cols, rows]; 2D -> output [rows, cols].
  *  shapes  : the block dim (and for 2D both dims) must be a multiple of 32;
- *            with RHT the RHT dim is the block dim.  Otherwise
- *            MXFP4_ERR_UNSUPPORTED_SHAPE.
+ *            with RHT the RHT dim is the block dim; for 1D blocks groups *
+ *            rows (and, along rows, groups * cols) must be below 2^31.
+ *            Otherwise MXFP4_ERR_UNSUPPORTED_SHAPE.
  *  2D with rht_d = 16 applies the RHT along the last dim before blocking;
  *  codes_t/scales_mma_t are then the codes of (W R)^T.
  * Passage: the abstract, which names hybrid 1D/2D blocks, the RHT and SR as
@@ -150,8 +151,8 @@ MXFP4_API mxfp4_status mxfp4_quantize(const void* in, int in_dtype, int64_t grou
  *  row_out, col_out : outputs of the two directions (codes_t/scales_mma_t
  *  must be NULL).  Every output equals, bit for bit, what the two separate
  *  mxfp4_quantize calls with these params write.
- *  shapes : rows % 32 == 0 and cols % 32 == 0, else
- *  MXFP4_ERR_UNSUPPORTED_SHAPE.
+ *  shapes : rows % 32 == 0, cols % 32 == 0, groups * rows < 2^31 and
+ *  groups * cols < 2^31, else MXFP4_ERR_UNSUPPORTED_SHAPE.
  * Passage: the abstract (hybrid 1D/2D blocks: activations and gradients enter
  * the forward/backward GEMMs along the contraction dim and the weight-gradient
  * GEMM along the token dim, the latter with the RHT). */

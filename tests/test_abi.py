@@ -118,3 +118,20 @@ def test_fused_gemm_host_validation_without_gpu(libpath):
     assert call(q=mxfp4.QuantOutputs(16, None, None, 16, None)) == -1      # 2D-only outputs given
     assert call(q=mxfp4.QuantOutputs(None, None, None, None, None)) == -1  # null codes
     assert "fused" in mxfp4.last_error()
+
+
+def test_index_range_is_checked_before_launch(libpath):
+    """The quantisers index rows and features of all groups in 32 bits:
+    2^31 rows are rejected on the host (no device memory is touched)."""
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    o = mxfp4.QuantOutputs(16, None, None, None, None)
+    for along in (0, 1):
+        p = mxfp4.QuantParams(mxfp4.BLOCK_1X32, along, 0, 0, 0, 0, 0)
+        assert L.mxfp4_quantize(ctypes.c_void_p(16), 0, 1, 1 << 31, 32, 32, ctypes.byref(p), ctypes.byref(o),
+                                None) == -2
+        assert "2^31" in mxfp4.last_error()
+    rp = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 0, 0, 0, 0, 0, 0)
+    cp = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0)
+    assert L.mxfp4_quantize_dual(ctypes.c_void_p(16), 0, 2, 1 << 30, 32, 32, ctypes.byref(rp), ctypes.byref(cp),
+                                 ctypes.byref(o), ctypes.byref(o), None) == -2
