@@ -95,6 +95,9 @@ struct Args {
     // (bf16 [M][ldy] and codes [M][N/2] leave through tensor maps)
     uint8_t* qscales;         // canonical [M][N/32], may be null
     uint8_t* qscales_mma;     // tensor-core layout of the [M, N/32] scales, may be null
+    int32_t q_sr;             // fused epilogue rounding: 0 nearest, 1 stochastic
+    uint32_t q_sr_offset;     // Philox counter word 2 of the fused codes (SR)
+    PhiloxKeys q_sr_keys;     // round keys of the fused codes' SR seed
 };
 
 struct Tile {

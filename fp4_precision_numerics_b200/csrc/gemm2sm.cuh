@@ -127,8 +127,9 @@ __device__ __forceinline__ Unit unit_info(const Args& a, const int32_t* s_off, c
 
 // FUSED (mode 0): the epilogue writes each output element as bf16 (round to
 // nearest even) and quantises every 32-column chunk of a row -- one lane's
-// registers -- as one 1x32 MXFP4 block of the bf16 values (nearest
-// rounding), i.e. exactly what mxfp4_quantize gives for the bf16 output.
+// registers -- as one 1x32 MXFP4 block of the bf16 values (nearest or
+// stochastic rounding), i.e. exactly what mxfp4_quantize gives for the bf16
+// output.
 template <bool FUSED>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -465,10 +466,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         y[2 * i + 1] = __fmul_rn(__uint_as_float(hb[i] & 0xFFFF0000u), inv);
                     }
                     uint32_t qb[4];
+                    if (a.q_sr) {
+                        // SR as mxfp4_quantize: element n = row * N + col of the
+                        // output, one Philox call per 16 elements, word w for
+                        // elements 4w..4w+3 of the 16
+                        const uint64_t gq = (uint64_t(row + lane) * uint64_t(a.N) + uint64_t(un.n0 + 32 * c)) >> 4;
+                        const Philox4 r0 = philox4x32_10(uint32_t(gq), uint32_t(gq >> 32), a.q_sr_offset, 0u,
+                                                         a.q_sr_keys);
+                        const Philox4 r1 = philox4x32_10(uint32_t(gq + 1), uint32_t((gq + 1) >> 32), a.q_sr_offset,
+                                                         0u, a.q_sr_keys);
+                        const uint32_t R[8] = {r0.w[0], r0.w[1], r0.w[2], r0.w[3], r1.w[0], r1.w[1], r1.w[2], r1.w[3]};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        qb[j] = e2m1x8_rn(y[8 * j], y[8 * j + 1], y[8 * j + 2], y[8 * j + 3], y[8 * j + 4],
-                                          y[8 * j + 5], y[8 * j + 6], y[8 * j + 7]);
+                        for (int j = 0; j < 4; ++j)
+                            qb[j] = e2m1x4_sr(y[8 * j], y[8 * j + 1], y[8 * j + 2], y[8 * j + 3], R[2 * j]) |
+                                    (e2m1x4_sr(y[8 * j + 4], y[8 * j + 5], y[8 * j + 6], y[8 * j + 7], R[2 * j + 1])
+                                     << 16);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            qb[j] = e2m1x8_rn(y[8 * j], y[8 * j + 1], y[8 * j + 2], y[8 * j + 3], y[8 * j + 4],
+                                              y[8 * j + 5], y[8 * j + 6], y[8 * j + 7]);
+                    }
                     if (lane == 0) bulk_wait_read<1>();
                     __syncwarp();
                     // staging: 32 rows x 64 B of bf16 in the 64-byte swizzle

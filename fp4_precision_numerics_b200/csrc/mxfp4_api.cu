@@ -317,6 +317,9 @@ struct FusedOut {
     uint8_t* codes;
     uint8_t* scales;
     uint8_t* scales_mma;
+    bool sr;
+    uint64_t sr_seed;
+    uint32_t sr_offset;
 };
 
 // Shared by the binary32-output and the fused (bf16 + MXFP4) entry points:
@@ -374,6 +377,9 @@ mxfp4_status grouped_gemm_impl(int op, int num_groups, const int32_t* group_offs
     a.status = status;
     if (f) {
         a.qscales = f->scales;
+        a.q_sr = f->sr ? 1 : 0;
+        a.q_sr_offset = f->sr_offset;
+        a.q_sr_keys = mxfp4::philox_keys(uint32_t(f->sr_seed), uint32_t(f->sr_seed >> 32));
         a.qscales_mma = f->scales_mma;
     }
 
@@ -731,13 +737,17 @@ mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t* group_off
 
 mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const int32_t* group_offsets, mxfp4_operand A,
                                       mxfp4_operand B, int64_t M, int64_t N, int64_t K, uint16_t* y, int64_t ldy,
-                                      const mxfp4_quant_outputs* q, void* stream) {
+                                      const mxfp4_quant_outputs* q, const mxfp4_quant_params* qp, void* stream) {
     if (op != MXFP4_GEMM_FPROP && op != MXFP4_GEMM_DGRAD)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: op must be FPROP or DGRAD");
     if (!y || !q || !q->codes)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: null output pointer");
     if (q->codes_t || q->scales_mma_t)
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: codes_t / scales_mma_t are for 2D blocks only");
+    if (qp && (qp->block != MXFP4_BLOCK_1X32 || qp->along_rows != 0 || qp->rht_d != 0 ||
+               (qp->rounding != MXFP4_ROUND_NEAREST && qp->rounding != MXFP4_ROUND_STOCHASTIC)))
+        return fail(MXFP4_ERR_INVALID_ARG,
+                    "mxfp4_grouped_gemm_fused: params must be 1x32 along the last dim, no RHT, RN or SR");
     if (N % 32 || K <= 0) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: N %% 32 != 0 or K <= 0");
     if (ldy < N) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_grouped_gemm_fused: ldy < N");
     if (ldy % 8) return fail(MXFP4_ERR_MISALIGNED, "mxfp4_grouped_gemm_fused: ldy must be a multiple of 8");
@@ -746,7 +756,8 @@ mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const int32_t* gro
     if (num_groups > mxfp4::gemm2::kMaxGroups || !pairs_enabled())
         return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_grouped_gemm_fused: at most %d groups, CTA pairs enabled",
                     mxfp4::gemm2::kMaxGroups);
-    FusedOut f{y, ldy, q->codes, q->scales, q->scales_mma};
+    const bool sr = qp && qp->rounding == MXFP4_ROUND_STOCHASTIC;
+    FusedOut f{y, ldy, q->codes, q->scales, q->scales_mma, sr, sr ? qp->sr_seed : 0u, sr ? qp->sr_offset : 0u};
     return grouped_gemm_impl(op, num_groups, group_offsets, A, B, M, N, K, nullptr, N, &f, stream);
 }
 

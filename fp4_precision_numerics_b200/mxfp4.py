@@ -85,7 +85,7 @@ def lib() -> ctypes.CDLL:
             L.mxfp4_grouped_gemm.argtypes = [st, st, vp, Operand, Operand, i64, i64, i64, vp, i64, vp]
             L.mxfp4_grouped_gemm.restype = st
             L.mxfp4_grouped_gemm_fused.argtypes = [st, st, vp, Operand, Operand, i64, i64, i64, vp, i64,
-                                                   ctypes.POINTER(QuantOutputs), vp]
+                                                   ctypes.POINTER(QuantOutputs), ctypes.POINTER(QuantParams), vp]
             L.mxfp4_grouped_gemm_fused.restype = st
             L.mxfp4_mma_scale_bytes.argtypes = [i64, i64]
             L.mxfp4_mma_scale_bytes.restype = ctypes.c_size_t
@@ -161,9 +161,9 @@ def mxfp4_grouped_gemm(op, num_groups, offsets_ptr, a: Operand, b: Operand, M, N
 
 
 def mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a: Operand, b: Operand, M, N, K, y_ptr, ldy,
-                             q: QuantOutputs, stream=None):
+                             q: QuantOutputs, qp: QuantParams | None = None, stream=None):
     _check(lib().mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a, b, M, N, K, y_ptr, ldy, ctypes.byref(q),
-                                          _stream(stream)))
+                                          ctypes.byref(qp) if qp is not None else None, _stream(stream)))
 
 
 def mxfp4_check_device_status(stream=None):
@@ -310,10 +310,11 @@ def grouped_gemm(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_codes,
 
 def grouped_gemm_fused(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_codes, b_scales_mma, M: int, N: int,
                        K: int, scales: bool = True, scales_mma: bool = True, y: torch.Tensor | None = None,
-                       out: dict | None = None, stream=None) -> tuple:
+                       out: dict | None = None, sr_seed=None, sr_offset: int = 0, stream=None) -> tuple:
     """FPROP/DGRAD with the fused epilogue: returns (y, q) with y the [M, N]
     bf16 output and q the dict ('codes', 'scales', 'scales_mma') of its
-    1x32-along-N MXFP4 quantisation with nearest rounding."""
+    1x32-along-N MXFP4 quantisation, nearest rounding or, with sr_seed,
+    stochastic rounding as quantize(y, sr_seed=..., sr_offset=...)."""
     assert offsets.dtype == torch.int32 and offsets.is_cuda
     G = offsets.numel() - 1
     dev = offsets.device
@@ -328,8 +329,10 @@ def grouped_gemm_fused(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_
     if scales_mma and "scales_mma" not in o:
         o["scales_mma"] = torch.empty((mxfp4_mma_scale_bytes(M, N // 32),), dtype=torch.uint8, device=dev)
     q = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")), None, None)
+    qp = QuantParams(BLOCK_1X32, 0, 0, 0, ROUND_STOCHASTIC if sr_seed is not None else ROUND_NEAREST,
+                     int(sr_seed or 0), int(sr_offset))
     mxfp4_grouped_gemm_fused(op, G, ctypes.c_void_p(offsets.data_ptr()),
                              Operand(a_codes.data_ptr(), a_scales_mma.data_ptr()),
                              Operand(b_codes.data_ptr(), b_scales_mma.data_ptr()), M, N, K,
-                             ctypes.c_void_p(y.data_ptr()), y.stride(0), q, stream)
+                             ctypes.c_void_p(y.data_ptr()), y.stride(0), q, qp, stream)
     return y, o

@@ -246,10 +246,12 @@ MXFP4_API mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t*
  *  - y: D rounded to bf16 (nearest even), [M, N] with row stride ldy
  *    elements (ldy >= N, ldy % 8 == 0), as raw bf16 bit patterns;
  *  - q->codes [M, N/2] and q->scales [M, N/32] / q->scales_mma (either may
- *    be null): the 1x32-along-N MXFP4 quantisation of y with nearest
- *    rounding, bit-identical to mxfp4_quantize(y, bf16, 1 group, M rows,
- *    N cols, ld = ldy) with no RHT and no SR.  q->codes_t / scales_mma_t
- *    must be null.
+ *    be null): the 1x32-along-N MXFP4 quantisation of y, bit-identical to
+ *    mxfp4_quantize(y, bf16, 1 group, M rows, N cols, ld = ldy) with the
+ *    params qp (NULL: nearest rounding).  qp must be 1x32 along the last
+ *    dim without RHT; its rounding is nearest or stochastic (sr_seed,
+ *    sr_offset as for mxfp4_quantize: element n = row * N + col).
+ *    q->codes_t / scales_mma_t must be null.
  * A, B, group_offsets, M, N, K as for mxfp4_grouped_gemm.  Needs the
  * CTA-pair kernel (G <= 255, not disabled by MXFP4_GEMM_CTA_PAIRS=0),
  * N % 32 == 0 and K > 0, else MXFP4_ERR_UNSUPPORTED_SHAPE.  Every 32-column
@@ -258,11 +260,11 @@ MXFP4_API mxfp4_status mxfp4_grouped_gemm(int op, int num_groups, const int32_t*
  * reaches HBM.
  * Passage: roboaidigest "What ALTO Actually Does" (activations take 1D
  * blocks; the next GEMM only ever sees quantised values) and the abstract
- * (hybrid 1D/2D block quantisation). */
+ * (hybrid 1D/2D block quantisation; SR on gradients, e.g. a dgrad output). */
 MXFP4_API mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const int32_t* group_offsets,
                                                 mxfp4_operand a, mxfp4_operand b, int64_t M, int64_t N, int64_t K,
                                                 uint16_t* y, int64_t ldy, const mxfp4_quant_outputs* q,
-                                                void* stream);
+                                                const mxfp4_quant_params* qp, void* stream);
 
 /* Copy the last error message of this thread into buf (NUL-terminated,
  * truncated to len).  Returns the message length. */

@@ -104,8 +104,9 @@ def test_fused_gemm_host_validation_without_gpu(libpath):
     q = mxfp4.QuantOutputs(16, None, None, None, None)
     off, y = ctypes.c_void_p(16), ctypes.c_void_p(16)
 
-    def call(op=0, G=1, M=128, N=192, K=128, y=y, ldy=192, q=q):
-        return L.mxfp4_grouped_gemm_fused(op, G, off, a, a, M, N, K, y, ldy, ctypes.byref(q), None)
+    def call(op=0, G=1, M=128, N=192, K=128, y=y, ldy=192, q=q, qp=None):
+        return L.mxfp4_grouped_gemm_fused(op, G, off, a, a, M, N, K, y, ldy, ctypes.byref(q),
+                                          ctypes.byref(qp) if qp is not None else None, None)
 
     assert call(op=mxfp4.GEMM_WGRAD) == -1                                  # wgrad has no fused epilogue
     assert call(y=None) == -1                                               # null y
@@ -117,6 +118,10 @@ def test_fused_gemm_host_validation_without_gpu(libpath):
     assert call(G=300) == -2                                                # CTA-pair kernel only
     assert call(q=mxfp4.QuantOutputs(16, None, None, 16, None)) == -1      # 2D-only outputs given
     assert call(q=mxfp4.QuantOutputs(None, None, None, None, None)) == -1  # null codes
+    assert call(qp=mxfp4.QuantParams(mxfp4.BLOCK_32X32, 0, 0, 0, 0, 0, 0)) == -1     # 2D blocks
+    assert call(qp=mxfp4.QuantParams(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0)) == -1      # along rows
+    assert call(qp=mxfp4.QuantParams(mxfp4.BLOCK_1X32, 0, 16, 1, 0, 0, 0)) == -1     # RHT
+    assert call(qp=mxfp4.QuantParams(mxfp4.BLOCK_1X32, 0, 0, 0, 9, 0, 0)) == -1      # bad rounding
     assert "fused" in mxfp4.last_error()
 
 

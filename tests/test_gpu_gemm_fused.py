@@ -1,5 +1,5 @@
 """GPU parity: the grouped GEMM with the fused epilogue (bf16 output plus its
-1x32-along-N MXFP4 quantisation, nearest rounding).
+1x32-along-N MXFP4 quantisation, nearest or stochastic rounding).
 
 Exact regime: operands on the E2M1 grid with block exponents in {-1, 0, 1}
 (every block holds a +-6 * 2^e entry, so quantisation is lossless) keep
@@ -53,7 +53,7 @@ def _offs_dev():
     return torch.tensor(OFFS.astype(np.int32), device="cuda")
 
 
-def _run(op, a_bits, w_bits):
+def _run(op, a_bits, w_bits, sr_seed=None, sr_offset=0):
     """Quantise (library) and run both epilogues; returns y fused, q, y fp32."""
     qa = mxfp4.quantize(dev_bf16(a_bits), scales=False, scales_mma=True)
     qw = mxfp4.quantize(dev_bf16(w_bits), block="32x32", scales=False, scales_mma=True, transposed=True)
@@ -61,7 +61,8 @@ def _run(op, a_bits, w_bits):
         b, bs, N, K = qw["codes"], qw["scales_mma"], NW, KW
     else:
         b, bs, N, K = qw["codes_t"], qw["scales_mma_t"], KW, NW
-    y, q = mxfp4.grouped_gemm_fused(op, _offs_dev(), qa["codes"], qa["scales_mma"], b, bs, M, N, K)
+    y, q = mxfp4.grouped_gemm_fused(op, _offs_dev(), qa["codes"], qa["scales_mma"], b, bs, M, N, K,
+                                    sr_seed=sr_seed, sr_offset=sr_offset)
     y32 = mxfp4.grouped_gemm(op, _offs_dev(), qa["codes"], qa["scales_mma"], b, bs, M, N, K)
     mxfp4.mxfp4_check_device_status()
     torch.cuda.synchronize()
@@ -125,3 +126,34 @@ def test_fused_epilogue_strided_output_leaves_padding():
     mxfp4.mxfp4_check_device_status()
     assert torch.equal(ybuf[:, NW:], torch.full((M, 64), 7.0, dtype=torch.bfloat16, device="cuda"))
     assert np.array_equal(_bits(ybuf[:, :NW].contiguous()), _bits(y32.to(torch.bfloat16)))
+
+
+def test_fused_epilogue_stochastic_rounding_exact_regime():
+    """SR codes of the dgrad output (a gradient): in the exact regime the
+    oracle's SR quantisation of its bf16-rounded binary64 product, bit for
+    bit (element n = row * N + col of the output, the given seed and offset)."""
+    op = mxfp4.GEMM_DGRAD
+    rng = np.random.default_rng(51)
+    a = _grid_blocks(rng, (M, NW), 1)
+    w = _grid_blocks(rng, (G, NW, KW), 32)
+    y, q, y32, N = _run(op, a, w, sr_seed=0x1234ABCD5678, sr_offset=17)
+    ref, _ = _oracle_product(op, a, w)
+    assert np.array_equal(host(y32).astype(np.float64), ref)
+    y_ref = oracle.bf16_round(ref)
+    c_ref, s_ref = oracle.quantize_1d(y_ref, sr=True, sr_seed=0x1234ABCD5678, sr_offset=17)
+    assert np.array_equal(_bits(y), y_ref)
+    assert np.array_equal(host(q["codes"]), c_ref)
+    assert np.array_equal(host(q["scales"]), s_ref)
+
+
+@pytest.mark.parametrize("op", [mxfp4.GEMM_FPROP, mxfp4.GEMM_DGRAD])
+def test_fused_epilogue_stochastic_rounding_matches_quantiser(op):
+    rng = np.random.default_rng(61 + op)
+    a = synth.bf16_bits(rng.standard_normal((M, NW if op == mxfp4.GEMM_DGRAD else KW)).astype(np.float32))
+    w = synth.bf16_bits((rng.standard_normal((G, NW, KW)) * 0.02).astype(np.float32))
+    y, q, y32, N = _run(op, a, w, sr_seed=7, sr_offset=3)
+    ql = mxfp4.quantize(y, sr_seed=7, sr_offset=3, scales=True, scales_mma=True)
+    assert torch.equal(q["codes"], ql["codes"][0])
+    assert torch.equal(q["scales"], ql["scales"][0])
+    rn = mxfp4.quantize(y, scales=False)
+    assert not torch.equal(q["codes"], rn["codes"][0]), "SR codes identical to nearest rounding"
