@@ -177,15 +177,19 @@ class Layer:
         """One training step.  `ev` (optional) maps a kernel name to a pair of
         CUDA events recorded around its launch on the current stream.  With
         `fused`, fprop and dgrad write bf16 outputs and their MXFP4
-        quantisation (the fused epilogue) instead of binary32."""
+        quantisation (the fused epilogue; SR for dgrad's gradient outputs)
+        instead of binary32."""
         mx = self.mx
         q = self.q
 
         def gemm(name, op, a, b, b_codes, b_scales, Mg, N, K, out):
             if fused:
+                # dgrad's output is a gradient: its codes take SR (own offsets)
                 y, qo = self.fused_out[name]
+                sr = dict(sr_seed=1, sr_offset=2000 + 2 * self.step_idx + (name == "dgrad_down")) \
+                    if op == mx.GEMM_DGRAD else {}
                 mx.grouped_gemm_fused(op, self.offsets, q[a]["codes"], q[a]["scales_mma"], q[b][b_codes],
-                                      q[b][b_scales], Mg, N, K, scales=False, y=y, out=qo)
+                                      q[b][b_scales], Mg, N, K, scales=False, y=y, out=qo, **sr)
             else:
                 mx.grouped_gemm(op, self.offsets, q[a]["codes"], q[a]["scales_mma"], q[b][b_codes], q[b][b_scales],
                                 Mg, N, K, out=out)
