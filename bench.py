@@ -252,12 +252,12 @@ class Layer:
 # 8-expert / 4096-token layer, whose every tensor is exactly a quarter of the
 # full one, times 4.  An entry must go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": 4 * (664.4e6 + 240.7e6), "deosc_down": 4 * (332.4e6 + 102.7e6),
-    "dual_x": 4 * (97.4e6 + 18.0e6), "dual_h": 4 * (97.4e6 + 14.5e6),
-    "dual_dy_up": 4 * (194.7e6 + 67.3e6), "dual_dy_down": 4 * (97.4e6 + 16.8e6),
-    "fprop_up": 4 * (97.3e6 + 334.3e6), "fprop_down": 4 * (61.3e6 + 138.7e6),
-    "dgrad_up": 4 * (122.6e6 + 153.4e6), "dgrad_down": 4 * (61.3e6 + 139.2e6),
-    "wgrad_up": 4 * (78.8e6 + 471.6e6), "wgrad_down": 4 * (51.9e6 + 206.2e6),
+    "deosc_up": 4 * (664.6e6 + 240.8e6), "deosc_down": 4 * (332.3e6 + 103.6e6),
+    "dual_x": 4 * (97.4e6 + 18.0e6), "dual_h": 4 * (97.4e6 + 16.1e6),
+    "dual_dy_up": 4 * (194.7e6 + 67.2e6), "dual_dy_down": 4 * (97.4e6 + 16.1e6),
+    "fprop_up": 4 * (97.0e6 + 333.7e6), "fprop_down": 4 * (61.3e6 + 139.5e6),
+    "dgrad_up": 4 * (122.6e6 + 153.2e6), "dgrad_down": 4 * (61.3e6 + 139.4e6),
+    "wgrad_up": 4 * (78.7e6 + 473.1e6), "wgrad_down": 4 * (51.9e6 + 206.7e6),
 }
 
 KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
