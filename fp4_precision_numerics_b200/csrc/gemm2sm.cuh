@@ -7,16 +7,21 @@
 //   - the pair owns two 128-row tiles of A of the same group (an m-tile
 //     pair; an odd last tile leaves the second half idle) and one 192-column
 //     tile of the output; each CTA stages its own 128 rows of A and its half
-//     (96 rows) of B, so per SM a K-step moves 28 KB instead of 40 KB and six
-//     stages fit in shared memory;
+//     (96 rows) of B.  A K-step is 512 elements (8 MMAs per barrier round):
+//     56 KB per CTA in three stages, A and B each in one TMA box through a
+//     [chunk][row][256 bytes] view of the codes (chunk stride 128 B);
 //   - the leader CTA's single MMA thread issues tcgen05.mma.cta_group::2
 //     (M = 256, N = 192, K = 64) over both CTAs' shared memory and tensor
 //     memory, and its commits are multicast to both CTAs' barriers;
 //   - the UE8M0 scales are staged per CTA by four loader warps with
 //     tcgen05.st, in the layout of a 128 x 256 one-CTA MMA (every CTA holds its
 //     own rows of A's scales and all of B's); the odd-tile offset of the
-//     192-wide B window is applied by the loaders, so each stage needs 20
-//     scale columns and two 192-column accumulators still fit in TMEM;
+//     192-wide B window is applied by the loaders, so a stage needs 40 scale
+//     columns and two 192-column accumulators still fit in TMEM.  The loaders
+//     arrive on the stage's full barrier, so the MMA thread waits once;
+//   - four epilogue warps drain the accumulator: binary32 output in 8 KB TMA
+//     stores (two 32-column chunks through a [column block][row][32 floats]
+//     view of D), or with FUSED the bf16 output and its 1x32 MXFP4 codes;
 //   - every wait is bounded; both CTAs meet at a cluster barrier before the
 //     pair's tensor memory is released.
 // No TMA multicast is used: every load reads global memory of this GPU into
