@@ -579,6 +579,26 @@ def run_reference(args):
 # ---------------------------------------------------------------------------
 # Main (our arm)
 # ---------------------------------------------------------------------------
+def fp4_mma_probe(mx, stream, mmas=16384, launches=10, warmup=3):
+    """The tensor pipe alone: the GEMM's own block-scaled MMA (M = 256,
+    N = 192, K = 64) issued back to back on operands resident in shared
+    memory (`mxfp4_mma_peak_probe`); median TFLOP/s of `launches` launches
+    after `warmup`, each timed with CUDA events on `stream`."""
+    import torch
+    for _ in range(warmup):
+        mx.mxfp4_mma_peak_probe(mmas, stream)
+    rates = []
+    for _ in range(launches):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        flops = mx.mxfp4_mma_peak_probe(mmas, stream)
+        e1.record(stream)
+        e1.synchronize()
+        rates.append(flops / (e0.elapsed_time(e1) / 1e3) / 1e12)
+    mx.mxfp4_check_device_status(stream)
+    return statistics.median(rates)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -781,6 +801,10 @@ def main():
                          "quantisations (2D de-oscillation W, SR dY, RHT-16 transposed operands); %.1f s on %d "
                          "threads of %d host cores" % (secs, threads, os.cpu_count() or 0)}
     ck = clocks.summary(t0, t1)
+    probe = fp4_mma_probe(layer.mx, stream)
+    if roof["bound"] == "tensor":
+        roof["peak_probe"] = probe
+        roof["frac_probe"] = roof["achieved"] / probe
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -794,6 +818,9 @@ def main():
         "quantise_frac_hbm_nominal": quant_gbs / NOMINAL_HBM_GBS,
         "gemm_frac_fp4_nominal": step_flops / (gemm_ms / 1e3) / 1e12 / NOMINAL_FP4_TFLOPS,
         "gemm_tflops": step_flops / (gemm_ms / 1e3) / 1e12, "gemm_frac_fp4": step_flops / (gemm_ms / 1e3) / 1e12 / fp4_peak,
+        "fp4_mma_probe": {"tflops": probe, "mmas_per_pair": 16384, "launches": 10,
+                          "what": "the GEMM's block-scaled MMA alone on resident operands, after the timed region"},
+        "gemm_frac_fp4_probe": step_flops / (gemm_ms / 1e3) / 1e12 / probe,
         "roofline": roof, "components": components,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d_bytes),
                 "d2h_bytes_per_step": int(d2h_bytes)},

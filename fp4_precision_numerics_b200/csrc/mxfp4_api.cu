@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemm2sm.cuh"
+#include "peak.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -759,6 +760,24 @@ mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const int32_t* gro
     const bool sr = qp && qp->rounding == MXFP4_ROUND_STOCHASTIC;
     FusedOut f{y, ldy, q->codes, q->scales, q->scales_mma, sr, sr ? qp->sr_seed : 0u, sr ? qp->sr_offset : 0u};
     return grouped_gemm_impl(op, num_groups, group_offsets, A, B, M, N, K, nullptr, N, &f, stream);
+}
+
+mxfp4_status mxfp4_mma_peak_probe(int64_t mmas_per_pair, double* flops, void* stream) {
+    if (mmas_per_pair < 1 || mmas_per_pair > (int64_t(1) << 22) || !flops)
+        return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_mma_peak_probe: mmas_per_pair must lie in [1, 2^22], flops non-null");
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_mma_peak_probe: no device status word");
+    if (cudaFuncSetAttribute(mxfp4::peak::mma_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             mxfp4::peak::kSmemBytes) != cudaSuccess)
+        return fail(MXFP4_ERR_CUDA, "mxfp4_mma_peak_probe: cannot raise the shared-memory limit");
+    const int64_t clusters = pair_clusters();
+    mxfp4::peak::mma_peak_kernel<<<unsigned(2 * clusters), mxfp4::peak::kThreads, mxfp4::peak::kSmemBytes,
+                                   static_cast<cudaStream_t>(stream)>>>(mmas_per_pair, status);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return fail(MXFP4_ERR_CUDA, "mxfp4_mma_peak_probe: launch failed: %s", cudaGetErrorString(e));
+    *flops = double(clusters) * double(mmas_per_pair) * 2.0 * 256.0 * 192.0 * 64.0;
+    return ok();
 }
 
 }  // extern "C"

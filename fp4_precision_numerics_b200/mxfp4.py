@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.mxfp4_grouped_gemm_fused.argtypes = [st, st, vp, Operand, Operand, i64, i64, i64, vp, i64,
                                                    ctypes.POINTER(QuantOutputs), ctypes.POINTER(QuantParams), vp]
             L.mxfp4_grouped_gemm_fused.restype = st
+            L.mxfp4_mma_peak_probe.argtypes = [i64, ctypes.POINTER(ctypes.c_double), vp]
+            L.mxfp4_mma_peak_probe.restype = st
             L.mxfp4_mma_scale_bytes.argtypes = [i64, i64]
             L.mxfp4_mma_scale_bytes.restype = ctypes.c_size_t
             L.mxfp4_last_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
@@ -164,6 +166,14 @@ def mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a: Operand, b: Operand
                              q: QuantOutputs, qp: QuantParams | None = None, stream=None):
     _check(lib().mxfp4_grouped_gemm_fused(op, num_groups, offsets_ptr, a, b, M, N, K, y_ptr, ldy, ctypes.byref(q),
                                           ctypes.byref(qp) if qp is not None else None, _stream(stream)))
+
+
+def mxfp4_mma_peak_probe(mmas_per_pair: int, stream=None) -> float:
+    """Launch the tensor-pipe peak probe on `stream`; returns the launch's
+    floating-point operations (the caller times the launch)."""
+    flops = ctypes.c_double(0.0)
+    _check(lib().mxfp4_mma_peak_probe(int(mmas_per_pair), ctypes.byref(flops), _stream(stream)))
+    return flops.value
 
 
 def mxfp4_check_device_status(stream=None):

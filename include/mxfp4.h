@@ -266,6 +266,20 @@ MXFP4_API mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const in
                                                 uint16_t* y, int64_t ldy, const mxfp4_quant_outputs* q,
                                                 const mxfp4_quant_params* qp, void* stream);
 
+/* Tensor-pipe peak probe, a measurement helper and not a step of the path:
+ * one CTA pair per two SMs (the grouped GEMM's launch shape) issues
+ * mmas_per_pair block-scaled MXFP4 MMAs of the GEMM's own shape (M = 256,
+ * N = 192, K = 64, UE8M0 scales) back to back on operands resident in shared
+ * memory, with no loads and no output.  Asynchronous on `stream`; the caller
+ * times the launch.  *flops (host) receives the launch's floating-point
+ * operations, 2 M N K per MMA.  Errors: MXFP4_ERR_INVALID_ARG unless
+ * 1 <= mmas_per_pair <= 2^22 and flops is non-null; MXFP4_ERR_CUDA if the
+ * launch fails; a wait that runs out sets MXFP4_ERR_DEVICE_TIMEOUT for
+ * mxfp4_check_device_status.
+ * Passage: none; it measures the FP4 roofline that the GEMMs are compared
+ * with, not an operation of the method. */
+MXFP4_API mxfp4_status mxfp4_mma_peak_probe(int64_t mmas_per_pair, double* flops, void* stream);
+
 /* Copy the last error message of this thread into buf (NUL-terminated,
  * truncated to len).  Returns the message length. */
 MXFP4_API size_t mxfp4_last_error(char* buf, size_t len);

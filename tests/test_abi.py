@@ -140,3 +140,16 @@ def test_index_range_is_checked_before_launch(libpath):
     cp = mxfp4.QuantParams(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0)
     assert L.mxfp4_quantize_dual(ctypes.c_void_p(16), 0, 2, 1 << 30, 32, 32, ctypes.byref(rp), ctypes.byref(cp),
                                  ctypes.byref(o), ctypes.byref(o), None) == -2
+
+
+def test_mma_peak_probe_host_validation_without_gpu(libpath):
+    """The peak probe rejects an MMA count outside [1, 2^22] and a null
+    result pointer before any CUDA call."""
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    f = ctypes.c_double(-1.0)
+    for n in (0, -5, (1 << 22) + 1):
+        assert L.mxfp4_mma_peak_probe(n, ctypes.byref(f), None) == -1
+    assert L.mxfp4_mma_peak_probe(16, None, None) == -1
+    assert "mmas_per_pair" in mxfp4.last_error()
+    assert f.value == -1.0
