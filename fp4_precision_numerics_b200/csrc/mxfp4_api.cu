@@ -5,7 +5,10 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <string>
 
 #include "../../include/mxfp4.h"
@@ -48,19 +51,33 @@ int num_sms() {
 }
 
 // CTAs of a persistent kernel that fit on the device at once (every SM
-// filled to its occupancy limit), cached per kernel; at least one per SM.
+// filled to its occupancy limit), at least one per SM.  Cached per (kernel,
+// block size, shared memory, device) under a lock: kernels of one signature
+// may differ in registers and hence occupancy.
+int64_t resident_ctas_of(const void* kern, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, int, size_t, int>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    const auto key = std::make_tuple(kern, threads, smem, dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto it = cache.find(key);
+        if (it != cache.end()) return int64_t(num_sms()) * it->second;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = 1;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = n;
+    return int64_t(num_sms()) * n;
+}
+
 template <typename K>
 int64_t resident_ctas(K kern, int threads, size_t smem) {
-    static int per_sm = 0;
-    if (per_sm <= 0) {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess || n <= 0) {
-            cudaGetLastError();
-            n = 1;
-        }
-        per_sm = n;
-    }
-    return int64_t(num_sms()) * per_sm;
+    return resident_ctas_of(reinterpret_cast<const void*>(kern), threads, smem);
 }
 
 // The pair GEMM's binary32 epilogue stores two 32-column chunks per TMA box.
@@ -69,10 +86,11 @@ constexpr bool kEpiPairStores = true;
 // Clusters of two CTAs of the pair GEMM that can be resident at once (one
 // CTA per SM; an SM left without a partner in its GPC stays idle).
 int pair_clusters() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return num_sms() / 2;
-    if (cached[dev] > 0) return cached[dev];
+    const int c = cached[dev].load();
+    if (c > 0) return c;
     int n = 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * unsigned(num_sms() / 2), 1, 1);
