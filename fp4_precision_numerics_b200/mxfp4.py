@@ -187,6 +187,62 @@ def version() -> str:
 # ---------------------------------------------------------------------------
 # Tensor helpers
 # ---------------------------------------------------------------------------
+def _require(cond: bool, msg: str) -> None:
+    """Argument checks of the tensor helpers.  They raise (and survive
+    `python -O`): a wrong dtype, layout or size would otherwise reach the
+    library as a pointer and become an out-of-bounds device access."""
+    if not cond:
+        raise ValueError(msg)
+
+
+def _check_buf(t, nbytes: int, name: str, dtype=torch.uint8) -> None:
+    """`t` is a contiguous CUDA tensor of `dtype` holding at least `nbytes`."""
+    _require(isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous(),
+             "%s: a contiguous CUDA %s tensor is required" % (name, dtype))
+    have = t.numel() * t.element_size()
+    _require(have >= nbytes, "%s: %d bytes, at least %d required" % (name, have, nbytes))
+
+
+def _check_input(x: torch.Tensor, name: str = "x") -> torch.Tensor:
+    if isinstance(x, torch.Tensor) and x.dim() == 2:
+        x = x.unsqueeze(0)
+    _require(isinstance(x, torch.Tensor) and x.is_cuda and x.dim() == 3 and x.stride(2) == 1,
+             "%s: a [rows, cols] or [groups, rows, cols] CUDA tensor with unit column stride is required" % name)
+    _require(x.dtype in (torch.bfloat16, torch.float32), "%s: bf16 or float32 required" % name)
+    _require(x.shape[0] == 1 or x.stride(0) == x.shape[1] * x.stride(1), "%s: groups must be back to back" % name)
+    return x
+
+
+def _check_offsets(offsets) -> None:
+    _require(isinstance(offsets, torch.Tensor) and offsets.is_cuda and offsets.dtype == torch.int32
+             and offsets.dim() == 1 and offsets.is_contiguous() and offsets.numel() >= 1,
+             "offsets: a contiguous 1D int32 CUDA tensor of G + 1 entries")
+
+
+def _check_quant_outputs(o: dict, G: int, Ro: int, Co: int, two_d: bool, R: int, C: int) -> None:
+    """Sizes of a quantiser's output buffers (those present in `o`): codes
+    [G, Ro, Co/2]; scales [G, Ro, Co/32] (2D: [G, R/32, C/32]); tensor-core
+    scales per group; for 2D the transpose's codes [G, C, R/2] and scales."""
+    _check_buf(o["codes"], G * Ro * (Co // 2), "codes")
+    if o.get("scales") is not None:
+        _check_buf(o["scales"], G * ((R // 32) * (C // 32) if two_d else Ro * (Co // 32)), "scales")
+    if o.get("scales_mma") is not None:
+        _check_buf(o["scales_mma"], G * mxfp4_mma_scale_bytes(Ro, Co // 32), "scales_mma")
+    if o.get("codes_t") is not None:
+        _check_buf(o["codes_t"], G * C * (R // 2), "codes_t")
+    if o.get("scales_mma_t") is not None:
+        _check_buf(o["scales_mma_t"], G * mxfp4_mma_scale_bytes(C, R // 32), "scales_mma_t")
+
+
+def _check_operands(op: int, G: int, M: int, N: int, K: int, a_codes, a_scales, b_codes, b_scales) -> None:
+    """Sizes of the GEMM operands as include/mxfp4.h lays them out."""
+    _check_buf(a_codes, M * K // 2, "a_codes")
+    _check_buf(a_scales, mxfp4_mma_scale_bytes(M, K // 32), "a_scales_mma")
+    groups_b = 1 if op == GEMM_WGRAD else G
+    _check_buf(b_codes, groups_b * N * K // 2, "b_codes")
+    _check_buf(b_scales, groups_b * mxfp4_mma_scale_bytes(N, K // 32), "b_scales_mma")
+
+
 def quantize(x: torch.Tensor, block: str = "1x32", along_rows: bool = False, rht_seed=None, sr_seed=None,
              sr_offset: int = 0, scales: bool = True, scales_mma: bool = False, transposed: bool = False,
              out: dict | None = None, stream=None) -> dict:
@@ -195,10 +251,7 @@ def quantize(x: torch.Tensor, block: str = "1x32", along_rows: bool = False, rht
     Returns a dict with 'codes', and as requested 'scales' (canonical),
     'scales_mma', 'codes_t' and 'scales_mma_t' (2D: the transpose's codes
     and tensor-core scales).  `out` may supply preallocated tensors."""
-    if x.dim() == 2:
-        x = x.unsqueeze(0)
-    assert x.is_cuda and x.dim() == 3 and x.stride(2) == 1
-    assert x.shape[0] == 1 or x.stride(0) == x.shape[1] * x.stride(1), "groups must be back to back"
+    x = _check_input(x)
     G, R, C = x.shape
     ld = x.stride(1)
     two_d = block == "32x32"
@@ -220,6 +273,7 @@ def quantize(x: torch.Tensor, block: str = "1x32", along_rows: bool = False, rht
             o["codes_t"] = torch.empty((G, C, R // 2), dtype=torch.uint8, device=dev)
         if scales_mma and "scales_mma_t" not in o:
             o["scales_mma_t"] = torch.empty((G, mxfp4_mma_scale_bytes(C, R // 32)), dtype=torch.uint8, device=dev)
+    _check_quant_outputs(o, G, Ro, Co, two_d, R, C)
     outs = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")),
                         _ptr(o.get("codes_t")), _ptr(o.get("scales_mma_t")))
     mxfp4_quantize(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), G, R, C, ld, p, outs, stream)
@@ -233,10 +287,7 @@ def quantize_dual(x: torch.Tensor, row_rht_seed=None, col_rht_seed=None, sr_seed
     in both 1D directions from one read: returns (row, col), the outputs of
     quantize(x, ...) along the last dim and quantize(x, along_rows=True, ...),
     each a dict like quantize's."""
-    if x.dim() == 2:
-        x = x.unsqueeze(0)
-    assert x.is_cuda and x.dim() == 3 and x.stride(2) == 1
-    assert x.shape[0] == 1 or x.stride(0) == x.shape[1] * x.stride(1), "groups must be back to back"
+    x = _check_input(x)
     G, R, C = x.shape
     rounding = ROUND_STOCHASTIC if sr_seed is not None else ROUND_NEAREST
     rp = QuantParams(BLOCK_1X32, 0, 16 if row_rht_seed is not None else 0, int(row_rht_seed or 0), rounding,
@@ -252,6 +303,7 @@ def quantize_dual(x: torch.Tensor, row_rht_seed=None, col_rht_seed=None, sr_seed
             o["scales"] = torch.empty((G, Ro, Co // 32), dtype=torch.uint8, device=dev)
         if scales_mma and "scales_mma" not in o:
             o["scales_mma"] = torch.empty((G, mxfp4_mma_scale_bytes(Ro, Co // 32)), dtype=torch.uint8, device=dev)
+        _check_quant_outputs(o, G, Ro, Co, False, R, C)
         outs.append(o)
     ro, co = outs
     qo_r = QuantOutputs(ro["codes"].data_ptr(), _ptr(ro.get("scales")), _ptr(ro.get("scales_mma")), None, None)
@@ -262,7 +314,8 @@ def quantize_dual(x: torch.Tensor, row_rht_seed=None, col_rht_seed=None, sr_seed
 
 
 def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, stream=None) -> torch.Tensor:
-    assert x.is_cuda and x.dim() == 2 and x.stride(1) == 1
+    _require(isinstance(x, torch.Tensor) and x.is_cuda and x.dim() == 2 and x.stride(1) == 1
+             and x.dtype in (torch.bfloat16, torch.float32), "x: a 2D bf16/float32 CUDA tensor with unit column stride")
     R, C = x.shape
     y = torch.empty((R, C), dtype=out_dtype, device=x.device)
     mxfp4_rht(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), R, C, x.stride(0), 16, int(seed),
@@ -273,12 +326,12 @@ def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, stream=None) -> tor
 def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_threshold: int = 4,
                  reset_period: int = 0, scales: bool = True, scales_mma: bool = False, transposed: bool = False,
                  out: dict | None = None, stream=None, freeze_lower: bool = False) -> dict:
-    if master.dim() == 2:
+    if isinstance(master, torch.Tensor) and master.dim() == 2:
         master = master.unsqueeze(0)
-    assert master.dtype == torch.float32 and master.stride(-1) == 1
-    assert master.shape[0] == 1 or master.stride(0) == master.shape[1] * master.shape[2]
-    assert master.stride(1) == master.shape[2]
-    assert state.dtype == torch.uint8 and state.is_contiguous() and state.numel() == master.numel()
+    _require(isinstance(master, torch.Tensor) and master.is_cuda and master.dtype == torch.float32
+             and master.dim() == 3 and master.is_contiguous(), "master: a contiguous float32 CUDA tensor")
+    _check_buf(state, master.numel(), "state")
+    _require(state.numel() == master.numel(), "state: one byte per weight")
     G, R, C = master.shape
     o = dict(out or {})
     dev = master.device
@@ -293,6 +346,7 @@ def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_thre
             o["codes_t"] = torch.empty((G, C, R // 2), dtype=torch.uint8, device=dev)
         if scales_mma and "scales_mma_t" not in o:
             o["scales_mma_t"] = torch.empty((G, mxfp4_mma_scale_bytes(C, R // 32)), dtype=torch.uint8, device=dev)
+    _check_quant_outputs(o, G, R, C, True, R, C)
     outs = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")),
                         _ptr(o.get("codes_t")), _ptr(o.get("scales_mma_t")))
     mxfp4_deosc_update(ctypes.c_void_p(master.data_ptr()), G, R, C, int(step),
@@ -305,12 +359,20 @@ def deosc_update(master: torch.Tensor, step: int, state: torch.Tensor, flip_thre
 def grouped_gemm(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_codes, b_scales_mma, M: int, N: int,
                  K: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """FPROP/DGRAD: out [M, N]; WGRAD: out [G, M, N] (see include/mxfp4.h)."""
-    assert offsets.dtype == torch.int32 and offsets.is_cuda
+    _check_offsets(offsets)
     G = offsets.numel() - 1
     if out is None:
         shape = (G, M, N) if op == GEMM_WGRAD else (M, N)
         out = torch.empty(shape, dtype=torch.float32, device=offsets.device)
+    _require(isinstance(out, torch.Tensor) and out.is_cuda and out.dtype == torch.float32 and out.stride(-1) == 1,
+             "out: a float32 CUDA tensor with unit column stride")
     ldo = out.stride(-2)
+    if op == GEMM_WGRAD:
+        _require(out.dim() == 3 and out.shape[0] >= G and out.shape[1] == M and out.shape[2] >= N
+                 and (G <= 1 or out.stride(0) == M * ldo), "out: [G, M, >= N] with group stride M * row stride")
+    else:
+        _require(out.dim() == 2 and out.shape[0] >= M and out.shape[1] >= N, "out: [>= M, >= N]")
+    _check_operands(op, G, M, N, K, a_codes, a_scales_mma, b_codes, b_scales_mma)
     mxfp4_grouped_gemm(op, G, ctypes.c_void_p(offsets.data_ptr()),
                        Operand(a_codes.data_ptr(), a_scales_mma.data_ptr()),
                        Operand(b_codes.data_ptr(), b_scales_mma.data_ptr()), M, N, K,
@@ -325,12 +387,15 @@ def grouped_gemm_fused(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_
     bf16 output and q the dict ('codes', 'scales', 'scales_mma') of its
     1x32-along-N MXFP4 quantisation, nearest rounding or, with sr_seed,
     stochastic rounding as quantize(y, sr_seed=..., sr_offset=...)."""
-    assert offsets.dtype == torch.int32 and offsets.is_cuda
+    _check_offsets(offsets)
     G = offsets.numel() - 1
     dev = offsets.device
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    assert y.dtype == torch.bfloat16 and y.stride(-1) == 1
+    _require(isinstance(y, torch.Tensor) and y.is_cuda and y.dtype == torch.bfloat16 and y.dim() == 2
+             and y.stride(-1) == 1 and y.shape[0] >= M and y.shape[1] >= N,
+             "y: a [>= M, >= N] bf16 CUDA tensor with unit column stride")
+    _check_operands(op, G, M, N, K, a_codes, a_scales_mma, b_codes, b_scales_mma)
     o = dict(out or {})
     if "codes" not in o:
         o["codes"] = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
@@ -338,6 +403,7 @@ def grouped_gemm_fused(op: int, offsets: torch.Tensor, a_codes, a_scales_mma, b_
         o["scales"] = torch.empty((M, N // 32), dtype=torch.uint8, device=dev)
     if scales_mma and "scales_mma" not in o:
         o["scales_mma"] = torch.empty((mxfp4_mma_scale_bytes(M, N // 32),), dtype=torch.uint8, device=dev)
+    _check_quant_outputs(o, 1, M, N, False, M, N)
     q = QuantOutputs(o["codes"].data_ptr(), _ptr(o.get("scales")), _ptr(o.get("scales_mma")), None, None)
     qp = QuantParams(BLOCK_1X32, 0, 0, 0, ROUND_STOCHASTIC if sr_seed is not None else ROUND_NEAREST,
                      int(sr_seed or 0), int(sr_offset))

@@ -189,7 +189,9 @@ def test_bad_group_offsets_flag_the_device_status():
 
 
 def test_host_rejects_bad_shapes_without_launch():
-    z = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    # buffers large enough for the claimed shapes, so the library's shape
+    # checks (not the binding's size checks) are what rejects the calls
+    z = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
     offs = _offsets_dev([0, 128])
     with pytest.raises(mxfp4.MXFP4Error) as e:
         mxfp4.grouped_gemm(mxfp4.GEMM_FPROP, offs, z, z, z, z, 128, 192, 100)   # K % 64
@@ -197,3 +199,27 @@ def test_host_rejects_bad_shapes_without_launch():
     with pytest.raises(mxfp4.MXFP4Error) as e:
         mxfp4.grouped_gemm(mxfp4.GEMM_FPROP, offs, z, z, z, z, 100, 192, 128)   # M % 128
     assert e.value.status == -2
+
+
+def test_binding_rejects_undersized_or_mistyped_buffers():
+    """The tensor helpers check dtype, layout and size before any call: an
+    undersized operand or a wrong-dtype output raises ValueError instead of
+    reaching the library as a pointer."""
+    offs = _offsets_dev([0, 128])
+    small = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        mxfp4.grouped_gemm(mxfp4.GEMM_FPROP, offs, small, small, small, small, 128, 192, 128)
+    big = torch.zeros(1 << 20, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ValueError):
+        mxfp4.grouped_gemm(mxfp4.GEMM_FPROP, offs, big, big, big, big, 128, 192, 128,
+                           out=torch.zeros((128, 192), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        mxfp4.grouped_gemm(mxfp4.GEMM_WGRAD, offs, big, big, big, big, 192, 192, 128,
+                           out=torch.zeros((1, 96, 192), dtype=torch.float32, device="cuda"))
+    x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        mxfp4.quantize(x, out={"codes": small})
+    with pytest.raises(ValueError):
+        mxfp4.quantize(x.float().t(), scales=False)          # column stride != 1
+    torch.cuda.synchronize()
+    mxfp4.mxfp4_check_device_status()
