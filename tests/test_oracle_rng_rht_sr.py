@@ -178,3 +178,16 @@ def test_sr_unbiased_over_1e6_draws():
             p = (float(v) - lo) / (hi - lo)
             sigma = (hi - lo) * np.sqrt(p * (1 - p) / n)
             assert abs(deq.mean() - float(v)) <= 5 * sigma + (hi - lo) * 2.0 ** -16
+
+
+def test_philox_known_answer_vectors():
+    """The oracle's Philox4x32-10 reproduces the published known-answer
+    vectors (tests/golden/philox4x32_10_kat.txt, cited there): an input of
+    all zeros, all ones and the digits of pi."""
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "philox4x32_10_kat.txt")
+    rows = [ln.split() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    assert len(rows) == 3
+    for r in rows:
+        w = [int(v, 16) for v in r]
+        assert [int(v) for v in oracle.philox4x32_10(w[0:4], w[4:6])] == w[6:10]
