@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 
 import oracle
+from fp4_precision_numerics_b200 import synth
 
 
 def e2m1_decode_bits(code: int) -> float:
@@ -174,3 +175,21 @@ def test_bf16_round_rounds_once_from_binary64():
              2.0 ** -134 + 2.0 ** -160: 0x0001, 2.0 ** -134: 0x0000}
     got = oracle.bf16_round(np.array(list(cases), dtype=np.float64))
     assert [int(g) for g in got] == list(cases.values())
+
+
+def test_operand_footprint_is_a_quarter_of_bf16():
+    """roboaidigest "What ALTO Actually Does": E2M1 values with per-block
+    UE8M0 scales give a theoretical 4x smaller operand than BF16.  The
+    oracle's packing: two codes per byte (exactly a quarter of the bf16
+    bytes), plus one scale byte per 32 elements (4.25 bits per element, a
+    16/4.25 = 3.76x reduction with scales; 1/1024 byte per element for the
+    32x32 weight blocks)."""
+    rng = np.random.default_rng(3)
+    x = synth.bf16_bits(rng.standard_normal((64, 256)).astype(np.float32))
+    codes, scales = oracle.quantize_1d(x)
+    assert codes.dtype == np.uint8 and scales.dtype == np.uint8
+    assert codes.nbytes * 4 == x.nbytes
+    assert (codes.nbytes + scales.nbytes) * 8 == x.size * 4.25
+    assert abs(x.nbytes / (codes.nbytes + scales.nbytes) - 16 / 4.25) < 1e-12
+    c2, s2 = oracle.quantize_2d(x)
+    assert c2.nbytes * 4 == x.nbytes and s2.nbytes * 1024 == x.size
