@@ -153,3 +153,72 @@ def test_mma_peak_probe_host_validation_without_gpu(libpath):
     assert L.mxfp4_mma_peak_probe(16, None, None) == -1
     assert "mmas_per_pair" in mxfp4.last_error()
     assert f.value == -1.0
+
+
+def test_every_host_check_returns_its_status(libpath):
+    """Each host-side check of include/mxfp4.h returns its documented status
+    before any CUDA call (pointers are fake, aligned or not as the case
+    needs; nothing is dereferenced on the host)."""
+    from fp4_precision_numerics_b200 import mxfp4
+    L = mxfp4.lib()
+    INV, SHAPE, ALIGN = -1, -2, -3
+    P = lambda *a: mxfp4.QuantParams(*a)
+    ok_p = P(mxfp4.BLOCK_1X32, 0, 0, 0, 0, 0, 0)
+    outs = mxfp4.QuantOutputs(16, None, None, None, None)
+
+    def quant(in_ptr=16, dtype=0, G=1, R=64, C=64, ld=64, p=ok_p, o=outs):
+        return L.mxfp4_quantize(ctypes.c_void_p(in_ptr), dtype, G, R, C, ld, ctypes.byref(p), ctypes.byref(o), None)
+
+    assert quant(dtype=7) == INV                                             # in_dtype
+    assert quant(ld=32) == INV                                               # ld < cols
+    assert quant(p=P(5, 0, 0, 0, 0, 0, 0)) == INV                            # block
+    assert quant(p=P(mxfp4.BLOCK_1X32, 0, 8, 1, 0, 0, 0)) == INV             # rht_d
+    assert quant(p=P(mxfp4.BLOCK_32X32, 0, 0, 0, 0, 0, 0), R=48) == SHAPE    # 2D rows % 32
+    assert quant(p=P(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0), R=48) == SHAPE     # along rows, rows % 32
+    assert quant(o=mxfp4.QuantOutputs(24, None, None, None, None)) == ALIGN  # codes misaligned
+    assert quant(o=mxfp4.QuantOutputs(16, None, None, 16, None)) == INV      # codes_t with 1D blocks
+    assert quant(p=P(mxfp4.BLOCK_32X32, 0, 0, 0, 0, 0, 0),
+                 o=mxfp4.QuantOutputs(16, None, None, None, 16)) == INV      # scales_mma_t without codes_t
+    assert quant(G=0) == 0 and quant(R=0) == 0                               # empty: nothing to do
+
+    rp, cp = ok_p, P(mxfp4.BLOCK_1X32, 1, 0, 0, 0, 0, 0)
+
+    def dual(R=64, C=64, r=rp, c=cp, in_ptr=16):
+        return L.mxfp4_quantize_dual(ctypes.c_void_p(in_ptr), 0, 1, R, C, C, ctypes.byref(r), ctypes.byref(c),
+                                     ctypes.byref(outs), ctypes.byref(outs), None)
+
+    assert dual(c=P(mxfp4.BLOCK_32X32, 1, 0, 0, 0, 0, 0)) == INV             # 2D blocks
+    assert dual(c=P(mxfp4.BLOCK_1X32, 1, 8, 1, 0, 0, 0)) == INV              # rht_d
+    sr = mxfp4.ROUND_STOCHASTIC
+    assert dual(r=P(mxfp4.BLOCK_1X32, 0, 0, 0, sr, 1, 0), c=P(mxfp4.BLOCK_1X32, 1, 0, 0, sr, 2, 0)) == INV  # seeds
+    assert dual(R=48) == SHAPE and dual(C=48) == SHAPE                       # multiples of 32
+    assert dual(in_ptr=18) == ALIGN                                          # input misaligned
+
+    def rht(in_ptr=16, out_ptr=16, dtype=0, out_dtype=1, R=4, C=32, ld=32):
+        return L.mxfp4_rht(ctypes.c_void_p(in_ptr), dtype, R, C, ld, 16, 1, ctypes.c_void_p(out_ptr), out_dtype, None)
+
+    assert rht(dtype=5) == INV and rht(out_dtype=5) == INV                   # dtypes
+    assert rht(C=24, ld=24) == SHAPE                                         # cols % 16
+    assert rht(out_ptr=20) == ALIGN                                          # output misaligned
+
+    def deosc(thr=4, freeze_lower=0, R=64, C=64, master=16):
+        d = mxfp4.DeoscParams(thr, 0, freeze_lower)
+        return L.mxfp4_deosc_update(ctypes.c_void_p(master), 1, R, C, 1, ctypes.byref(d), ctypes.c_void_p(16),
+                                    ctypes.byref(outs), None)
+
+    assert deosc(thr=0) == INV and deosc(thr=8) == INV                       # threshold in 1..7
+    assert deosc(freeze_lower=2) == INV
+    assert deosc(R=48) == SHAPE and deosc(C=40) == SHAPE                     # 32x32 blocks
+    assert deosc(master=8) == ALIGN
+
+    A = mxfp4.Operand(16, 16)
+
+    def gemm(op=0, G=1, M=128, N=192, K=128, ldo=192, out=16, a=A):
+        return L.mxfp4_grouped_gemm(op, G, ctypes.c_void_p(16), a, a, M, N, K, ctypes.c_void_p(out), ldo, None)
+
+    assert gemm(N=0) == INV and gemm(ldo=100) == INV                         # geometry, ldo < N
+    assert gemm(G=5000) == SHAPE                                             # group count
+    assert gemm(op=mxfp4.GEMM_WGRAD, K=192) == SHAPE                         # wgrad tokens % 128
+    assert gemm(K=96) == SHAPE and gemm(M=192) == SHAPE                      # K % 64, M % 128
+    assert gemm(ldo=194) == ALIGN                                            # ldo % 4
+    assert gemm(out=24) == ALIGN and gemm(a=mxfp4.Operand(16, 40)) == ALIGN  # pointer alignment
