@@ -16,6 +16,7 @@
 #include "gemm.cuh"
 #include "gemm2sm.cuh"
 #include "peak.cuh"
+#include "selftest.cuh"
 #include "quantize.cuh"
 
 namespace {
@@ -796,6 +797,13 @@ mxfp4_status mxfp4_mma_peak_probe(int64_t mmas_per_pair, double* flops, void* st
         return fail(MXFP4_ERR_CUDA, "mxfp4_mma_peak_probe: launch failed: %s", cudaGetErrorString(e));
     *flops = double(clusters) * double(mmas_per_pair) * 2.0 * 256.0 * 192.0 * 64.0;
     return ok();
+}
+
+mxfp4_status mxfp4_selftest_wait_timeout(void* stream) {
+    uint32_t* status = status_word();
+    if (!status) return fail(MXFP4_ERR_CUDA, "mxfp4_selftest_wait_timeout: no device status word");
+    mxfp4::selftest::wait_timeout_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(status);
+    return check_launch("mxfp4_selftest_wait_timeout");
 }
 
 }  // extern "C"

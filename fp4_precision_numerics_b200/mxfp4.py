@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.mxfp4_grouped_gemm_fused.restype = st
             L.mxfp4_mma_peak_probe.argtypes = [i64, ctypes.POINTER(ctypes.c_double), vp]
             L.mxfp4_mma_peak_probe.restype = st
+            L.mxfp4_selftest_wait_timeout.argtypes = [vp]
+            L.mxfp4_selftest_wait_timeout.restype = st
             L.mxfp4_mma_scale_bytes.argtypes = [i64, i64]
             L.mxfp4_mma_scale_bytes.restype = ctypes.c_size_t
             L.mxfp4_last_error.argtypes = [ctypes.c_char_p, ctypes.c_size_t]
@@ -174,6 +176,12 @@ def mxfp4_mma_peak_probe(mmas_per_pair: int, stream=None) -> float:
     flops = ctypes.c_double(0.0)
     _check(lib().mxfp4_mma_peak_probe(int(mmas_per_pair), ctypes.byref(flops), _stream(stream)))
     return flops.value
+
+
+def mxfp4_selftest_wait_timeout(stream=None):
+    """Launch the failure-detection self-test (a bounded wait that expires
+    after about 2 s); read its result with mxfp4_check_device_status."""
+    _check(lib().mxfp4_selftest_wait_timeout(_stream(stream)))
 
 
 def mxfp4_check_device_status(stream=None):

@@ -280,6 +280,18 @@ MXFP4_API mxfp4_status mxfp4_grouped_gemm_fused(int op, int num_groups, const in
  * with, not an operation of the method. */
 MXFP4_API mxfp4_status mxfp4_mma_peak_probe(int64_t mmas_per_pair, double* flops, void* stream);
 
+/* Self-test of failure detection, not a step of the path: one small kernel
+ * in which a thread waits, through the same bounded wait as every pipeline
+ * role, on a barrier that nothing completes.  When the wait budget (2 s)
+ * runs out it records a timeout for the "mma" role in the device status word
+ * and sets its CTA's abort flag, which ends a second thread's wait (started
+ * 50 ms later) without a second record; the kernel then returns and the
+ * context stays usable.  A following mxfp4_check_device_status() returns
+ * MXFP4_ERR_DEVICE_TIMEOUT naming that role only.  Asynchronous on
+ * `stream`.  Errors: MXFP4_ERR_CUDA if the launch fails.
+ * Passage: none; it checks the library's own failure detection. */
+MXFP4_API mxfp4_status mxfp4_selftest_wait_timeout(void* stream);
+
 /* Copy the last error message of this thread into buf (NUL-terminated,
  * truncated to len).  Returns the message length. */
 MXFP4_API size_t mxfp4_last_error(char* buf, size_t len);
