@@ -56,6 +56,30 @@ def load_peaks():
 # ---------------------------------------------------------------------------
 # Workload
 # ---------------------------------------------------------------------------
+def algorithmic_work(rows_real, M, n_experts):
+    """Per-launch algorithmic work of the step's kernels, the roofline
+    numerators.  GEMMs: 2 r N K FLOP over the r real (routed) rows.  The dual
+    quantiser reads its bf16 input once and writes codes (1/2 B) and scales
+    (1/32 B) in each direction: 3.0625 B per element of the padded [M, cols]
+    input.  De-oscillation reads the fp32 master and the state byte and
+    writes the state, the W and W^T codes and both scale layouts: 7.0625 B
+    per weight."""
+    r = rows_real
+    gemm_flops = {
+        "fprop_up": 2.0 * r * F * D, "fprop_down": 2.0 * r * D * D,
+        "dgrad_up": 2.0 * r * F * D, "dgrad_down": 2.0 * r * D * D,
+        "wgrad_up": 2.0 * r * F * D, "wgrad_down": 2.0 * r * D * D,
+    }
+    q2 = 2.0 + 2 * (0.5 + 1.0 / 32)
+    per_weight = 4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32
+    quant_bytes = {
+        "deosc_up": n_experts * F * D * per_weight,
+        "deosc_down": n_experts * D * D * per_weight,
+        "dual_x": M * D * q2, "dual_h": M * D * q2, "dual_dy_up": M * F * q2, "dual_dy_down": M * D * q2,
+    }
+    return gemm_flops, quant_bytes
+
+
 class Layer:
     """Device buffers of one MoE layer replica and its training step."""
 
@@ -121,21 +145,7 @@ class Layer:
         self.dw_down = torch.empty((E, D, D), **f32)
         self.step_idx = 0
         self.launches_per_step = 12
-        # algorithmic work
-        r = self.rows_real
-        self.gemm_flops = {
-            "fprop_up": 2.0 * r * F * D, "fprop_down": 2.0 * r * D * D,
-            "dgrad_up": 2.0 * r * F * D, "dgrad_down": 2.0 * r * D * D,
-            "wgrad_up": 2.0 * r * F * D, "wgrad_down": 2.0 * r * D * D,
-        }
-        # quantise bytes: the dual quantiser reads its bf16 input once and writes
-        # codes (1/2 B) + scales (1/32 B) in each direction; de-osc adds state r/w
-        q2 = 2.0 + 2 * (0.5 + 1.0 / 32)
-        self.quant_bytes = {
-            "deosc_up": E * F * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
-            "deosc_down": E * D * D * (4 + 1 + 1 + 0.5 + 0.5 + 2.0 / 32),
-            "dual_x": M * D * q2, "dual_h": M * D * q2, "dual_dy_up": M * F * q2, "dual_dy_down": M * D * q2,
-        }
+        self.gemm_flops, self.quant_bytes = algorithmic_work(self.rows_real, M, E)
         self.gemm_dims = {
             "fprop_up": (M, F, D), "fprop_down": (M, D, D), "dgrad_up": (M, D, F), "dgrad_down": (M, D, D),
             "wgrad_up": (F, D, M), "wgrad_down": (D, D, M),
