@@ -204,3 +204,42 @@ def test_grouped_gemm_segments():
     offs = [0, 4, 4, 10]
     C = oracle.grouped_gemm_f64(A, B, offs)
     assert np.allclose(C[:4], A[:4] @ B[0].T) and np.allclose(C[4:], A[4:] @ B[2].T)
+
+
+def test_oracle_is_unchanged_at_O0():
+    """The C oracle built at -O0 gives the same bits as the -O2 build on every
+    step (RHT, 1D/2D quantisation with RN and SR, the transposed layout,
+    de-oscillation over three steps, the binary64 GEMM loop): no result
+    depends on undefined behaviour, uninitialised memory or optimisation."""
+    import os
+    import subprocess
+
+    def run_all():
+        rng = np.random.default_rng(11)
+        x = synth.bf16_bits((rng.standard_normal((64, 96)) * 3).astype(np.float32))
+        out = [oracle.rht_rows(x, 5)]
+        out += list(oracle.quantize_1d(x, rht_d=16, rht_seed=5, sr=True, sr_seed=9, sr_offset=2))
+        out += list(oracle.quantize_1d_transposed(x, rht_d=16, rht_seed=5, sr=True, sr_seed=9, sr_offset=3))
+        out += list(oracle.quantize_2d(x))
+        m = (rng.standard_normal((2, 64, 64)) * 0.02).astype(np.float32)
+        st = np.zeros(m.shape, dtype=np.uint8)
+        for step in range(3):
+            out += list(oracle.deosc_update(m + np.float32(1e-3 * step), step, st))
+            out.append(st.copy())
+        A, B = rng.standard_normal((8, 64)), rng.standard_normal((5, 64))
+        out.append(oracle.gemm_f64_loop(A, B))
+        return out
+
+    ref = run_all()
+    so0 = os.path.join(oracle._BUILD, "libmxfp4_oracle_O0.so")
+    subprocess.check_call(["gcc", "-O0", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC",
+                           "-shared", "-o", so0, oracle._SRC, "-lm"])
+    saved = (oracle._SO, oracle._lib)
+    try:
+        oracle._SO, oracle._lib = so0, None
+        got = run_all()
+    finally:
+        oracle._SO, oracle._lib = saved
+    assert len(got) == len(ref)
+    for a, b in zip(ref, got):
+        assert a.dtype == b.dtype and np.array_equal(a.view(np.uint8), b.view(np.uint8))
