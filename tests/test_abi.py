@@ -222,3 +222,34 @@ def test_every_host_check_returns_its_status(libpath):
     assert gemm(K=96) == SHAPE and gemm(M=192) == SHAPE                      # K % 64, M % 128
     assert gemm(ldo=194) == ALIGN                                            # ldo % 4
     assert gemm(out=24) == ALIGN and gemm(a=mxfp4.Operand(16, 40)) == ALIGN  # pointer alignment
+
+
+C_CONSUMER = r'''
+#include "mxfp4.h"
+#include <stdio.h>
+int main(void) {
+    mxfp4_quant_params p = {0};
+    mxfp4_quant_outputs o = {0};
+    char msg[256];
+    int st = mxfp4_quantize(NULL, MXFP4_DTYPE_BF16, 1, 32, 32, 32, &p, &o, NULL);
+    mxfp4_last_error(msg, sizeof msg);
+    printf("%s|%zu|%d|%s\n", mxfp4_version(), mxfp4_mma_scale_bytes(128, 4), st, msg);
+    return 0;
+}
+'''
+
+
+def test_header_is_plain_c_and_a_c_program_uses_the_library(libpath):
+    """include/mxfp4.h is a C ABI: it compiles as strict C99, and a C program
+    links against libmxfp4.so and calls it (version, a layout helper and a
+    host-side check; none needs a GPU)."""
+    d = os.path.join(ROOT, "tests", "_build")
+    os.makedirs(d, exist_ok=True)
+    src, exe = os.path.join(d, "c_consumer.c"), os.path.join(d, "c_consumer")
+    with open(src, "w") as f:
+        f.write(C_CONSUMER)
+    libdir = os.path.dirname(libpath)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    src, "-o", exe, "-L", libdir, "-lmxfp4", "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.strip().split("|")
+    assert "sm_100a" in out[0] and out[1] == "512" and out[2] == "-1" and "null" in out[3]
