@@ -253,3 +253,21 @@ def test_header_is_plain_c_and_a_c_program_uses_the_library(libpath):
                     src, "-o", exe, "-L", libdir, "-lmxfp4", "-Wl,-rpath," + libdir], check=True)
     out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.strip().split("|")
     assert "sm_100a" in out[0] and out[1] == "512" and out[2] == "-1" and "null" in out[3]
+
+
+def test_tensor_core_scale_layout_is_a_bijection(libpath):
+    """The tensor-core scale layout of include/mxfp4.h (the decoder the GPU
+    tests use) sends distinct (row, scale) pairs to distinct bytes inside
+    mxfp4_mma_scale_bytes(R, S), and fills that buffer exactly when R and S
+    are whole chunks (128 rows x 4 scales)."""
+    import numpy as np
+    from fp4_precision_numerics_b200 import mxfp4
+    from tests.gpu_util import mma_scales_to_rows
+    for R, S in ((128, 4), (256, 8), (2880, 90), (200, 5), (33, 3), (67584, 180)):
+        size = mxfp4.mxfp4_mma_scale_bytes(R, S)
+        assert size == ((R + 127) // 128) * ((S + 3) // 4) * 512
+        off = mma_scales_to_rows(np.arange(size, dtype=np.int64), R, S)
+        assert off.shape == (R, S) and off.min() >= 0 and off.max() < size
+        assert len(np.unique(off)) == R * S
+        if R % 128 == 0 and S % 4 == 0:
+            assert R * S == size
