@@ -25,6 +25,16 @@ thread_local std::string g_last_error;
 
 __device__ uint32_t g_device_status;
 
+// Snapshots of the status word taken by mxfp4_check_device_status: each
+// check reads and clears the word in one atomic exchange on the caller's
+// stream and leaves the value it took in its own slot, so checks running at
+// the same time on different streams or threads do not overwrite each
+// other's result (up to kStatusSlots concurrent checks).
+constexpr uint32_t kStatusSlots = 64;
+__device__ uint32_t g_status_taken[kStatusSlots];
+
+__global__ void status_take_kernel(uint32_t slot) { g_status_taken[slot] = atomicExch(&g_device_status, 0u); }
+
 mxfp4_status fail(mxfp4_status st, const char* fmt, ...) {
     char buf[512];
     va_list ap;
@@ -553,15 +563,18 @@ size_t mxfp4_last_error(char* buf, size_t len) {
 }
 
 mxfp4_status mxfp4_check_device_status(void* stream) {
+    static std::atomic<uint32_t> next_slot{0};
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint32_t slot = next_slot.fetch_add(1u) % kStatusSlots;
     uint32_t v = 0;
-    cudaError_t e = cudaMemcpyFromSymbolAsync(&v, g_device_status, sizeof(v), 0, cudaMemcpyDeviceToHost, st);
+    status_take_kernel<<<1, 1, 0, st>>>(slot);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        e = cudaMemcpyFromSymbolAsync(&v, g_status_taken, sizeof(v), sizeof(uint32_t) * slot, cudaMemcpyDeviceToHost,
+                                      st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return fail(MXFP4_ERR_CUDA, "check_device_status: %s", cudaGetErrorString(e));
     if (v == 0) return ok();
-    const uint32_t zero = 0;
-    e = cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, st);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (v & mxfp4::kStatusTimeout)
         return fail(MXFP4_ERR_DEVICE_TIMEOUT, "device wait timed out (status 0x%08x: roles %s%s%s%s%s)", v,
                     (v & mxfp4::kRoleProducer) ? "producer " : "", (v & mxfp4::kRoleMma) ? "mma " : "",
@@ -685,21 +698,38 @@ mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t groups, i
                                         : launch_dual<float>(qa, cp->rht_d == 16, rp->rht_d == 16, sr, st);
 }
 
-mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int d, uint64_t seed,
-                       void* out, int out_dtype, void* stream) {
+mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int axis, int d,
+                       uint64_t seed, void* out, int out_dtype, void* stream) {
     if (!in || !out) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: null pointer");
+    if (axis != 0 && axis != 1) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: axis must be 0 or 1");
     if (d != 16) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: only d = 16 is supported");
     if ((in_dtype != MXFP4_DTYPE_BF16 && in_dtype != MXFP4_DTYPE_F32) ||
         (out_dtype != MXFP4_DTYPE_BF16 && out_dtype != MXFP4_DTYPE_F32))
         return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: bad dtype");
     if (rows < 0 || cols < 0 || ld < cols) return fail(MXFP4_ERR_INVALID_ARG, "mxfp4_rht: bad geometry");
-    if (cols % 16) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_rht: cols %% 16 != 0");
+    if (axis == 1 && cols % 16) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_rht: cols %% 16 != 0");
+    if (axis == 0 && rows % 16) return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_rht(axis 0): rows %% 16 != 0");
     const int esz = in_dtype == MXFP4_DTYPE_BF16 ? 2 : 4;
     if (!aligned16(in) || !aligned16(out) || (ld * esz) % 16)
         return fail(MXFP4_ERR_MISALIGNED, "mxfp4_rht: pointers/rows not 16-byte aligned");
     if (rows == 0 || cols == 0) return ok();
     const uint32_t signs = rht_sign_mask(seed);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (axis == 0) {
+        const unsigned grid = grid_for((rows / 16) * cols, 256);
+        if (in_dtype == MXFP4_DTYPE_BF16) {
+            if (out_dtype == MXFP4_DTYPE_BF16)
+                mxfp4::rht_dim0_kernel<uint16_t, true><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(in), rows, cols, ld, signs, out);
+            else
+                mxfp4::rht_dim0_kernel<uint16_t, false><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(in), rows, cols, ld, signs, out);
+        } else {
+            if (out_dtype == MXFP4_DTYPE_BF16)
+                mxfp4::rht_dim0_kernel<float, true><<<grid, 256, 0, st>>>(static_cast<const float*>(in), rows, cols, ld, signs, out);
+            else
+                mxfp4::rht_dim0_kernel<float, false><<<grid, 256, 0, st>>>(static_cast<const float*>(in), rows, cols, ld, signs, out);
+        }
+        return check_launch("mxfp4_rht(axis 0)");
+    }
     const unsigned grid = grid_for(rows * (cols / 16), 256);
     if (in_dtype == MXFP4_DTYPE_BF16) {
         if (out_dtype == MXFP4_DTYPE_BF16)

@@ -161,16 +161,26 @@ MXFP4_API mxfp4_status mxfp4_quantize_dual(const void* in, int in_dtype, int64_t
                                  const mxfp4_quant_params* col_params, const mxfp4_quant_outputs* row_out,
                                  const mxfp4_quant_outputs* col_out, void* stream);
 
-/* Standalone randomized Hadamard transform along the last dim, d = 16:
- * out[r, :] = RHT(in[r, :]) in the butterfly order stated above.
+/* Standalone randomized Hadamard transform, d = 16, in the butterfly order
+ * stated above, with the signs of `seed`.
+ *  axis 1: along the last dim, out[r, 16j:16j+16] = RHT(in[r, 16j:16j+16]);
+ *          cols % 16 == 0.
+ *  axis 0: along dim 0 (the token dim of the weight-gradient operands),
+ *          out[16j:16j+16, c] = RHT(in[16j:16j+16, c]); rows % 16 == 0.
+ *          This is the transform the along-rows quantisation applies before
+ *          blocking, here with the output kept in the input's layout.
  *  in  : device [rows, cols] (row stride ld elements), bf16 or f32.
  *  out : device [rows, cols] contiguous, out_dtype F32 (bit contract) or
- *        BF16 (round-to-nearest-even of the F32 result).
- *  cols % 16 == 0.
+ *        BF16 (round-to-nearest-even of the F32 result; a NaN stays a NaN,
+ *        its payload unspecified).
+ *  Errors: MXFP4_ERR_INVALID_ARG for a null pointer, a bad dtype or axis, or
+ *  d != 16; MXFP4_ERR_UNSUPPORTED_SHAPE when the transformed dim is not a
+ *  multiple of 16; MXFP4_ERR_MISALIGNED for pointers or rows not 16-byte
+ *  aligned.
  * Passage: the abstract, which lists randomized Hadamard transforms among the
  * recipe's techniques. */
-MXFP4_API mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int d,
-                       uint64_t seed, void* out, int out_dtype, void* stream);
+MXFP4_API mxfp4_status mxfp4_rht(const void* in, int in_dtype, int64_t rows, int64_t cols, int64_t ld, int axis,
+                                 int d, uint64_t seed, void* out, int out_dtype, void* stream);
 
 /* De-oscillation parameters. */
 typedef struct {
@@ -296,9 +306,17 @@ MXFP4_API mxfp4_status mxfp4_selftest_wait_timeout(void* stream);
  * truncated to len).  Returns the message length. */
 MXFP4_API size_t mxfp4_last_error(char* buf, size_t len);
 
-/* Synchronise `stream`, read and clear the device status word of the
- * current device.  Returns MXFP4_OK, MXFP4_ERR_DEVICE_TIMEOUT or
- * MXFP4_ERR_DEVICE_BAD_INPUT (details via mxfp4_last_error). */
+/* Read and clear the device status word of the current device, then
+ * synchronise `stream`.  Returns MXFP4_OK, MXFP4_ERR_DEVICE_TIMEOUT or
+ * MXFP4_ERR_DEVICE_BAD_INPUT (details via mxfp4_last_error), or
+ * MXFP4_ERR_CUDA if the read itself fails.
+ * The word is one per device, shared by every stream and every call of this
+ * library in the process.  The check takes it with one atomic exchange
+ * (read and clear in a single step), issued on `stream` after the work
+ * already queued there, so no recorded bit is lost.  It does not wait for
+ * work on other streams: a status that a kernel on another stream records
+ * is reported by whichever check runs next, on whatever stream, so it can
+ * be attributed to the wrong stream when calls overlap. */
 MXFP4_API mxfp4_status mxfp4_check_device_status(void* stream);
 
 /* Library version string. */
