@@ -967,8 +967,17 @@ __global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __g
 }
 
 // ---------------------------------------------------------------------------
-// Standalone RHT along the last dim: one thread per 16-element chunk.
+// Standalone RHT.  bf16 output: round-to-nearest-even of the binary32 result
+// by cvt.rn.bf16x2.f32 (a NaN stays a NaN, infinities and overflow give
+// infinities).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Along the last dim: one thread per 16-element chunk of a row.
 template <typename InT, bool OUT_BF16>
 __global__ void __launch_bounds__(256) rht_kernel(const InT* __restrict__ in, int64_t rows, int64_t cols, int64_t ld,
                                                   uint32_t signs, void* __restrict__ out) {
@@ -984,12 +993,7 @@ __global__ void __launch_bounds__(256) rht_kernel(const InT* __restrict__ in, in
         if constexpr (OUT_BF16) {
             uint32_t w[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t lo = __float_as_uint(x[2 * k]), hi = __float_as_uint(x[2 * k + 1]);
-                const uint32_t rlo = (lo + 0x7FFFu + ((lo >> 16) & 1u)) >> 16;
-                const uint32_t rhi = (hi + 0x7FFFu + ((hi >> 16) & 1u)) >> 16;
-                w[k] = rlo | (rhi << 16);
-            }
+            for (int k = 0; k < 8; ++k) w[k] = bf16x2_rn(x[2 * k], x[2 * k + 1]);
             uint4* o = reinterpret_cast<uint4*>(static_cast<uint16_t*>(out) + row * cols + col0);
             o[0] = make_uint4(w[0], w[1], w[2], w[3]);
             o[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -997,6 +1001,37 @@ __global__ void __launch_bounds__(256) rht_kernel(const InT* __restrict__ in, in
             float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + row * cols + col0);
 #pragma unroll
             for (int k = 0; k < 4; ++k) o[k] = make_float4(x[4 * k], x[4 * k + 1], x[4 * k + 2], x[4 * k + 3]);
+        }
+    }
+}
+
+// Along dim 0: one thread per (16-row chunk, column).  Consecutive threads
+// take consecutive columns, so every load and store of a warp covers one
+// contiguous row segment.  The output keeps the input's [rows, cols] layout.
+template <typename InT, bool OUT_BF16>
+__global__ void __launch_bounds__(256) rht_dim0_kernel(const InT* __restrict__ in, int64_t rows, int64_t cols,
+                                                       int64_t ld, uint32_t signs, void* __restrict__ out) {
+    const int64_t total = (rows >> 4) * cols;
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t rb = i / cols;
+        const int64_t col = i - rb * cols;
+        const int64_t r0 = rb << 4;
+        float x[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if constexpr (sizeof(InT) == 2)
+                x[k] = __uint_as_float(uint32_t(__ldg(reinterpret_cast<const unsigned short*>(in) + (r0 + k) * ld + col)) << 16);
+            else
+                x[k] = __ldg(reinterpret_cast<const float*>(in) + (r0 + k) * ld + col);
+        }
+        rht16(x, signs);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            if constexpr (OUT_BF16)
+                static_cast<uint16_t*>(out)[(r0 + k) * cols + col] = uint16_t(bf16x2_rn(x[k], 0.0f) & 0xFFFFu);
+            else
+                static_cast<float*>(out)[(r0 + k) * cols + col] = x[k];
         }
     }
 }

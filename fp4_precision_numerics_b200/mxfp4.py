@@ -77,7 +77,7 @@ def lib() -> ctypes.CDLL:
                                               ctypes.POINTER(QuantParams), ctypes.POINTER(QuantOutputs),
                                               ctypes.POINTER(QuantOutputs), vp]
             L.mxfp4_quantize_dual.restype = st
-            L.mxfp4_rht.argtypes = [vp, st, i64, i64, i64, st, ctypes.c_uint64, vp, st, vp]
+            L.mxfp4_rht.argtypes = [vp, st, i64, i64, i64, st, st, ctypes.c_uint64, vp, st, vp]
             L.mxfp4_rht.restype = st
             L.mxfp4_deosc_update.argtypes = [vp, i64, i64, i64, ctypes.c_uint32, ctypes.POINTER(DeoscParams), vp,
                                              ctypes.POINTER(QuantOutputs), vp]
@@ -150,8 +150,8 @@ def mxfp4_quantize_dual(x_ptr, in_dtype, groups, rows, cols, ld, row_params: Qua
                                      _stream(stream)))
 
 
-def mxfp4_rht(x_ptr, in_dtype, rows, cols, ld, d, seed, out_ptr, out_dtype, stream=None):
-    _check(lib().mxfp4_rht(x_ptr, in_dtype, rows, cols, ld, d, seed, out_ptr, out_dtype, _stream(stream)))
+def mxfp4_rht(x_ptr, in_dtype, rows, cols, ld, axis, d, seed, out_ptr, out_dtype, stream=None):
+    _check(lib().mxfp4_rht(x_ptr, in_dtype, rows, cols, ld, axis, d, seed, out_ptr, out_dtype, _stream(stream)))
 
 
 def mxfp4_deosc_update(master_ptr, groups, rows, cols, step, params: DeoscParams, state_ptr,
@@ -321,12 +321,15 @@ def quantize_dual(x: torch.Tensor, row_rht_seed=None, col_rht_seed=None, sr_seed
     return ro, co
 
 
-def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, stream=None) -> torch.Tensor:
+def rht(x: torch.Tensor, seed: int, out_dtype=torch.float32, axis: int = 1, stream=None) -> torch.Tensor:
+    """RHT-16 of a 2D tensor along the last dim (axis 1) or along dim 0
+    (axis 0); the output keeps x's shape."""
     _require(isinstance(x, torch.Tensor) and x.is_cuda and x.dim() == 2 and x.stride(1) == 1
              and x.dtype in (torch.bfloat16, torch.float32), "x: a 2D bf16/float32 CUDA tensor with unit column stride")
+    _require(axis in (0, 1), "axis: 0 or 1")
     R, C = x.shape
     y = torch.empty((R, C), dtype=out_dtype, device=x.device)
-    mxfp4_rht(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), R, C, x.stride(0), 16, int(seed),
+    mxfp4_rht(ctypes.c_void_p(x.data_ptr()), _dtype_code(x), R, C, x.stride(0), int(axis), 16, int(seed),
               ctypes.c_void_p(y.data_ptr()), _dtype_code(y), stream)
     return y
 

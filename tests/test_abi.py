@@ -70,7 +70,7 @@ def test_host_validation_without_gpu(libpath):
     assert L.mxfp4_quantize(ctypes.c_void_p(16), 0, 1, 4, 32, 32, ctypes.byref(p), ctypes.byref(o), None) == -1
     assert "rounding" in mxfp4.last_error()
     # rht with unsupported d
-    assert L.mxfp4_rht(ctypes.c_void_p(16), 0, 4, 32, 32, 8, 0, ctypes.c_void_p(16), 1, None) == -1
+    assert L.mxfp4_rht(ctypes.c_void_p(16), 0, 4, 32, 32, 1, 8, 0, ctypes.c_void_p(16), 1, None) == -1
     # gemm: bad op, null operands
     a = mxfp4.Operand(None, None)
     assert L.mxfp4_grouped_gemm(7, 1, ctypes.c_void_p(16), a, a, 128, 192, 128, ctypes.c_void_p(16), 192, None) == -1
@@ -194,11 +194,15 @@ def test_every_host_check_returns_its_status(libpath):
     assert dual(R=48) == SHAPE and dual(C=48) == SHAPE                       # multiples of 32
     assert dual(in_ptr=18) == ALIGN                                          # input misaligned
 
-    def rht(in_ptr=16, out_ptr=16, dtype=0, out_dtype=1, R=4, C=32, ld=32):
-        return L.mxfp4_rht(ctypes.c_void_p(in_ptr), dtype, R, C, ld, 16, 1, ctypes.c_void_p(out_ptr), out_dtype, None)
+    def rht(in_ptr=16, out_ptr=16, dtype=0, out_dtype=1, R=4, C=32, ld=32, axis=1):
+        return L.mxfp4_rht(ctypes.c_void_p(in_ptr), dtype, R, C, ld, axis, 16, 1, ctypes.c_void_p(out_ptr), out_dtype,
+                           None)
 
     assert rht(dtype=5) == INV and rht(out_dtype=5) == INV                   # dtypes
-    assert rht(C=24, ld=24) == SHAPE                                         # cols % 16
+    assert rht(axis=2) == INV and rht(axis=-1) == INV                        # axis 0 or 1
+    assert rht(C=24, ld=24) == SHAPE                                         # cols % 16 along the last dim
+    assert rht(axis=0, R=24) == SHAPE                                        # rows % 16 along dim 0
+    assert rht(axis=0, R=4, C=24, ld=24) == SHAPE                            # (cols need not be)
     assert rht(out_ptr=20) == ALIGN                                          # output misaligned
 
     def deosc(thr=4, freeze_lower=0, R=64, C=64, master=16):

@@ -188,16 +188,67 @@ def test_2d_weights_and_transpose(rht, sr):
 
 
 # ----------------------------------------------------------- standalone RHT
-def test_rht_standalone():
+def _rht_ref(xh, seed, axis):
+    """Oracle RHT along the last dim, or along dim 0 as the oracle's RHT of the transpose."""
+    if axis == 1:
+        return oracle.rht_rows(xh, seed=seed)
+    return np.ascontiguousarray(oracle.rht_rows(np.ascontiguousarray(xh.T), seed=seed).T)
+
+
+def _bf16_out_matches(yb, ref):
+    """bf16 output against the oracle's nearest-even rounding of the binary32
+    result: bit-equal where the result is a number, a NaN where it is NaN."""
+    want = oracle.bf16_round(ref.astype(np.float64))
+    nan = np.isnan(ref)
+    got_nan = ((yb & 0x7F80) == 0x7F80) & ((yb & 0x7F) != 0)
+    return np.array_equal(yb[~nan], want[~nan]) and bool(got_nan[nan].all())
+
+
+@pytest.mark.parametrize("axis", [1, 0])
+def test_rht_standalone(axis):
+    """RHT-16 along either dim, binary32 and bf16 outputs, bf16 and binary32
+    inputs, a ragged tail (77 rows along the last dim; 320 columns, not a
+    multiple of the 256-thread block, along dim 0)."""
     rng = np.random.default_rng(12)
-    xf = rng.standard_normal((77, 320)).astype(np.float32)
+    shape = (77, 320) if axis == 1 else (96, 320)
+    xf = rng.standard_normal(shape).astype(np.float32)
     xb = synth.bf16_bits(xf)
     for xh, xd in ((xb, dev_bf16(xb)), (xf, dev_f32(xf))):
-        y = host(mxfp4.rht(xd, seed=21))
-        ref = oracle.rht_rows(xh, seed=21)
+        y = host(mxfp4.rht(xd, seed=21, axis=axis))
+        ref = _rht_ref(xh, 21, axis)
         assert np.array_equal(y.view(np.uint32), ref.view(np.uint32))
-        yb = host(mxfp4.rht(xd, seed=21, out_dtype=torch.bfloat16).view(torch.int16)).view(np.uint16)
-        assert np.array_equal(yb, synth.bf16_bits(ref))
+        yb = host(mxfp4.rht(xd, seed=21, out_dtype=torch.bfloat16, axis=axis).view(torch.int16)).view(np.uint16)
+        assert _bf16_out_matches(yb, ref)
+
+
+@pytest.mark.parametrize("axis", [1, 0])
+def test_rht_non_finite_and_overflow(axis):
+    """NaN and infinity propagate through the butterfly as the oracle's
+    binary32 arithmetic says, a NaN stays a NaN in the bf16 output, and
+    binary32 results past the largest bf16 round to infinity there."""
+    rng = np.random.default_rng(13)
+    x = rng.standard_normal((64, 64)).astype(np.float32)
+    x[3, 5] = np.nan
+    x[17, 40] = np.inf
+    x[30, 2] = -np.inf
+    # chunks x_i = s_i * c (s the RHT signs): output 0 of the chunk is exactly
+    # 16 c / 4 = 4c, the others 0.  4 * 0.8495e38 lies past the bf16 rounding
+    # edge to infinity (3.3961e38), 4 * 0.8472e38 just below the largest bf16
+    s = oracle.rht_signs(3)
+    for j, c in enumerate((0.8495e38, 0.8472e38)):
+        x[44, 16 * j:16 * j + 16] = (s * np.float32(c)).astype(np.float32)
+        x[16 * j:16 * j + 16, 50] = (s * np.float32(c)).astype(np.float32)
+    xd = dev_f32(x)
+    y = host(mxfp4.rht(xd, seed=3, axis=axis))
+    ref = _rht_ref(x, 3, axis)
+    nan = np.isnan(ref)
+    assert nan.any() and np.isinf(ref).any()
+    assert np.array_equal(np.isnan(y), nan)
+    assert np.array_equal(y[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    yb = host(mxfp4.rht(xd, seed=3, out_dtype=torch.bfloat16, axis=axis).view(torch.int16)).view(np.uint16)
+    assert _bf16_out_matches(yb, ref)
+    finite = np.isfinite(ref)
+    assert (np.abs(ref[finite]) >= 3.3961e38).any(), "no binary32 result rounds to a bf16 infinity"
 
 
 # ----------------------------------------------------------- de-oscillation
@@ -225,6 +276,62 @@ def test_deosc_steps_bit_exact(freeze_lower):
             assert np.array_equal(nibbles(host(out["codes_t"])[g]), nibbles(c_ref[g]).T)
     frozen = (st_ref >> 7).sum()
     assert frozen > 0                     # the boundary weights did oscillate and freeze
+
+
+@pytest.mark.parametrize("freeze_lower", [False, True])
+def test_deosc_resume_bit_exact(tmp_path, freeze_lower):
+    """Through the library: stop after step k, write the fp32 masters and
+    the state bytes to a file, read them into fresh device buffers and
+    continue.  Every later step's codes (W and W^T), scales and state equal
+    the uninterrupted run's and the oracle's; the reset period falls inside
+    the resumed part."""
+    G, R, C = 2, 256, 512
+    w0 = synth.deosc_master(groups=G, rows=R, cols=C, seed=7)
+    n_steps, k = 16, 7
+    kw = dict(flip_threshold=3, reset_period=10, freeze_lower=freeze_lower)
+
+    def upd(step):
+        return synth.deosc_update_noise(w0.shape, step, std=2e-4)
+
+    wd, st = dev_f32(w0), torch.zeros((G, R, C), dtype=torch.uint8, device="cuda")
+    w_ref, st_ref = w0.copy(), np.zeros((G, R, C), dtype=np.uint8)
+    run = []
+    for step in range(n_steps):
+        if step:
+            w_ref = (w_ref + upd(step)).astype(np.float32)
+            wd.copy_(dev_f32(w_ref))
+        out = mxfp4.deosc_update(wd, step, st, scales=True, transposed=True, **kw)
+        c_ref, s_ref = oracle.deosc_update(w_ref, step, st_ref, **kw)
+        torch.cuda.synchronize()
+        run.append({n: host(t).copy() for n, t in out.items() if n in ("codes", "scales", "codes_t")})
+        run[-1]["state"] = host(st).copy()
+        assert np.array_equal(run[-1]["codes"], c_ref) and np.array_equal(run[-1]["state"], st_ref), step
+    assert (run[k]["state"] >> 7).any(), "no weight froze before the checkpoint"
+    del wd, st
+
+    wd, st = dev_f32(w0), torch.zeros((G, R, C), dtype=torch.uint8, device="cuda")
+    w = w0.copy()
+    for step in range(k + 1):
+        if step:
+            w = (w + upd(step)).astype(np.float32)
+            wd.copy_(dev_f32(w))
+        mxfp4.deosc_update(wd, step, st, scales=True, transposed=True, **kw)
+    path = tmp_path / ("deosc_step%d.npz" % k)
+    np.savez(path, master=host(wd), state=host(st), step=k)
+    del wd, st
+    ck = np.load(path)
+    wd = dev_f32(ck["master"])
+    st = torch.from_numpy(ck["state"].copy()).cuda()
+    w = ck["master"].copy()
+    for step in range(int(ck["step"]) + 1, n_steps):
+        w = (w + upd(step)).astype(np.float32)
+        wd.copy_(dev_f32(w))
+        out = mxfp4.deosc_update(wd, step, st, scales=True, transposed=True, **kw)
+        torch.cuda.synchronize()
+        for n in ("codes", "scales", "codes_t"):
+            assert np.array_equal(host(out[n]), run[step][n]), (step, n)
+        assert np.array_equal(host(st), run[step]["state"]), step
+    mxfp4.mxfp4_check_device_status()
 
 
 def test_misaligned_rows_are_rejected():
