@@ -2,6 +2,7 @@
 the abstract), de-oscillation traces and binary64 GEMM.  Hand-worked
 examples, invariants and the textbook matrix product."""
 import numpy as np
+import pytest
 
 import oracle
 from fp4_precision_numerics_b200 import synth
@@ -243,3 +244,45 @@ def test_oracle_is_unchanged_at_O0():
     assert len(got) == len(ref)
     for a, b in zip(ref, got):
         assert a.dtype == b.dtype and np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+@pytest.mark.parametrize("freeze_lower", [False, True])
+def test_deosc_resume_equivalence(tmp_path, freeze_lower):
+    """The fp32 master weights and the one state byte per weight are the whole
+    de-oscillation state: stopping after step k, writing both to a file,
+    reading them back into fresh arrays and continuing gives, at every later
+    step, the same codes, scales and state as the run that never stopped
+    (the reset period falls inside the resumed part, so the step number is
+    carried too)."""
+    G, R, C = 2, 64, 96
+    w0 = synth.deosc_master(groups=G, rows=R, cols=C, seed=7)
+    n_steps, k, kw = 15, 7, dict(flip_threshold=3, reset_period=10, freeze_lower=freeze_lower)
+
+    def update(w, step):
+        return (w + synth.deosc_update_noise(w.shape, step, std=2e-4)).astype(np.float32)
+
+    w, st = w0.copy(), np.zeros((G, R, C), dtype=np.uint8)
+    ref = []
+    for step in range(n_steps):
+        if step:
+            w = update(w, step)
+        c, s = oracle.deosc_update(w, step, st, **kw)
+        ref.append((c, s, st.copy()))
+    assert (ref[-1][2] >> 7).any() and (ref[k][2] >> 7).any(), "no weight froze: the test would not exercise the state"
+
+    w, st = w0.copy(), np.zeros((G, R, C), dtype=np.uint8)
+    for step in range(k + 1):
+        if step:
+            w = update(w, step)
+        oracle.deosc_update(w, step, st, **kw)
+    path = tmp_path / ("deosc_step%d.npz" % k)
+    np.savez(path, master=w, state=st, step=k)
+    del w, st
+    ck = np.load(path)
+    w, st, k2 = ck["master"].copy(), ck["state"].copy(), int(ck["step"])
+    assert k2 == k
+    for step in range(k + 1, n_steps):
+        w = update(w, step)
+        c, s = oracle.deosc_update(w, step, st, **kw)
+        assert np.array_equal(c, ref[step][0]) and np.array_equal(s, ref[step][1]), step
+        assert np.array_equal(st, ref[step][2]), step

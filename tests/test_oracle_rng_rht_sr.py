@@ -191,3 +191,52 @@ def test_philox_known_answer_vectors():
     for r in rows:
         w = [int(v, 16) for v in r]
         assert [int(v) for v in oracle.philox4x32_10(w[0:4], w[4:6])] == w[6:10]
+
+
+# Largest |P(both round up) - P(first up) P(second up)| over every pair of
+# kept positions (F1, F2) for the two elements of a word that draw a 16-bit
+# value and its bit reversal (elements 4m, 4m+1 and 4m+2, 4m+3): 8.31e-5,
+# reached at F1 = F2 = 43691 (f = 2/3).  It is found by counting, for every
+# (F1, F2), the draws r in [0, 2^16) with F1 + r >= 2^16 and
+# F2 + reverse16(r) >= 2^16.  Elements drawing disjoint bytes are independent.
+SR_PAIR_DEPENDENCE_BOUND = 8.31e-5
+
+
+def test_sr_pair_decisions_are_nearly_independent():
+    """Joint behaviour of the SR decisions inside one Philox word, measured
+    through the oracle's quantiser over 2^20 blocks (one counter pair per
+    block): every element rounds up with frequency F/2^16, and every pair of
+    elements of a word rounds up together with frequency P1 P2 within the
+    layout's dependence bound (zero for elements on disjoint bytes) plus 5
+    standard deviations.  A layout that handed two elements the same or
+    overlapping random bits would fail: at f = 1/2 a shared draw gives a
+    joint frequency of 1/2 instead of 1/4."""
+    nb = 1 << 20
+    # block scale 2^0 (block max 6 at element 31); elements 0..27 sit in
+    # [1, 1.5) at kept positions F (value 1 + F/2^17, exact in binary32)
+    Fs = np.array([43691, 32768, 21845, 58982, 6554, 43691, 32768,
+                   16384, 49152, 43691, 21845, 32768, 65535, 1,
+                   43691, 43691, 32768, 32768, 21845, 43691, 5000,
+                   60000, 40000, 20000, 43691, 21845, 50000, 32768], dtype=np.int64)
+    row = np.zeros(32, dtype=np.float32)
+    row[:28] = (1.0 + Fs / 131072.0).astype(np.float32)
+    assert np.all(((row[:28].astype(np.float64) - 1.0) * 131072.0) == Fs)
+    row[31] = 6.0
+    x = np.broadcast_to(row, (nb, 32)).copy()
+    codes, scales = oracle.quantize_1d(x, sr=True, sr_seed=0xC0FFEE, sr_offset=11)
+    assert np.all(scales == 127)
+    nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(nb, 32)
+    assert np.all(np.isin(nib[:, :28], (2, 3)))
+    up = (nib[:, :28] == 3)
+    p = Fs / 65536.0
+    freq = up.mean(axis=0)
+    sig = np.sqrt(p * (1 - p) / nb)
+    assert np.all(np.abs(freq - p) <= 5 * sig + 1e-12), np.abs(freq - p) / np.maximum(sig, 1e-12)
+    for w in range(7):
+        for a, b in ((0, 1), (2, 3), (0, 2), (0, 3), (1, 2), (1, 3)):
+            i, j = 4 * w + a, 4 * w + b
+            q = p[i] * p[j]
+            joint = float(np.mean(up[:, i] & up[:, j]))
+            shared = (a, b) in ((0, 1), (2, 3))
+            bound = (SR_PAIR_DEPENDENCE_BOUND if shared else 0.0) + 5 * np.sqrt(max(q * (1 - q), 1e-12) / nb)
+            assert abs(joint - q) <= bound, (w, a, b, joint, q)
