@@ -188,6 +188,7 @@ class Layer:
         `fused`, fprop and dgrad write bf16 outputs and their MXFP4
         quantisation (the fused epilogue; SR for dgrad's gradient outputs)
         instead of binary32."""
+        import torch
         mx = self.mx
         q = self.q
 
@@ -204,8 +205,14 @@ class Layer:
                                 Mg, N, K, out=out)
 
         def rec(name, i):
+            # an NVTX range per launch (for profiler timelines) and, when
+            # asked, CUDA events around it
+            if i == 0:
+                torch.cuda.nvtx.range_push(name)
             if ev is not None:
                 ev[name][i].record()
+            if i == 1:
+                torch.cuda.nvtx.range_pop()
 
         s = self.step_idx
         rec("deosc_up", 0)
@@ -269,6 +276,21 @@ DRAM_BYTES_FULL = {
     "wgrad_up": 4 * (78.7e6 + 473.1e6), "wgrad_down": 4 * (51.9e6 + 206.7e6),
 }
 
+# Thread instructions per element of the stochastic-rounding quantisers:
+# ncu smsp__inst_executed.sum x 32 / elements of one launch (profiles/ gives
+# the commands).  An entry must go back to None when its kernel changes.
+SR_INST_PER_ELEMENT = {"dual_dy_up": 20.84, "dual_dy_down": 21.19, "rows_sr": 10.39}
+SMSP_PER_SM = 4          # warp schedulers per SM, each issuing one warp instruction per cycle
+
+
+def issue_roof_ms(inst_per_element, elements, n_sms, sm_mhz):
+    """Time to issue `inst_per_element` thread instructions for every element
+    at one warp instruction per scheduler per cycle on every SM at the given
+    clock: the ALU roof of an instruction-bound kernel."""
+    warp_inst = inst_per_element * elements / 32.0
+    return warp_inst / (n_sms * SMSP_PER_SM) / (sm_mhz * 1e6) * 1e3
+
+
 KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
            "dual_dy_down", "dgrad_down", "wgrad_up", "wgrad_down"]
 
@@ -283,9 +305,10 @@ class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
-    # NVML clock-event reason bits
-    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
-                   "hw_thermal_slowdown": 0x40}
+    # NVML clock-event reason bits (every one NVML defines, so a slow clock is never left unexplained)
+    REASON_BITS = {"gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+                   "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                   "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100}
 
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
@@ -353,6 +376,17 @@ class ClockSampler:
                 self.proc.kill()
         if self.thread is not None:
             self.thread.join(timeout=2)
+
+    def summary_windows(self, windows):
+        """Summary of the samples taken inside any of the (t0, t1) windows."""
+        rows = [r for r in self.samples if any(a <= r[0] <= b for a, b in windows)]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for r in rows:
+            reasons |= r[3]
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
+                "sm_mhz_min": min(r[1] for r in rows), "reasons": sorted(reasons), "samples": len(rows)}
 
     def summary(self, t0, t1):
         rows = [r for r in self.samples if t0 <= r[0] <= t1] or self.samples
@@ -517,20 +551,35 @@ def oracle_timing():
     return rep
 
 
-def quant_sweep(iters=20, warmup=3):
+def quant_sweep(iters=20, warmup=3, stream=None):
     """GPU timing of the 1x32 quantiser alone on the quantise-sweep shapes
     (bf16 Gaussian draws on the device -- the kernels' time does not depend
     on the values --, RHT-16, nearest and stochastic rounding):
     median of `iters` CUDA-event timings after `warmup`, with L2 flushed
     (a 256 MB write) before every timed launch.  Bytes per element: 2 in,
-    1/2 + 1/32 out."""
+    1/2 + 1/32 out.  The launch floor is the same measurement on a single
+    32 x 32 block (one CTA): what a launch costs with no data to move."""
     import numpy as np
     import torch
 
     from fp4_precision_numerics_b200 import mxfp4, synth
     peaks = load_peaks()
-    dev = torch.device("cuda", 0)
+    dev = torch.device("cuda", torch.cuda.current_device())
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(x, out, sr):
+        ts = []
+        for i in range(warmup + iters):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mxfp4.quantize(x, rht_seed=1, sr_seed=1 if sr else None, sr_offset=i, scales=True, out=out)
+            e1.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
     rows = []
     for (R, C) in synth.QUANT_SWEEP_SHAPES:
         g = torch.Generator(device=dev)
@@ -539,24 +588,20 @@ def quant_sweep(iters=20, warmup=3):
         out = dict(codes=torch.empty((1, R, C // 2), dtype=torch.uint8, device=dev),
                    scales=torch.empty((1, R, C // 32), dtype=torch.uint8, device=dev))
         for sr in (False, True):
-            ts = []
-            for i in range(warmup + iters):
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                mxfp4.quantize(x, rht_seed=1, sr_seed=1 if sr else None, sr_offset=i, scales=True, out=out)
-                e1.record()
-                torch.cuda.synchronize()
-                if i >= warmup:
-                    ts.append(e0.elapsed_time(e1))
-            ms = float(np.median(ts))
+            ms = timed(x, out, sr)
             gbs = R * C * (2 + 0.5 + 1.0 / 32) / (ms / 1e3) / 1e9
             rows.append({"shape": [R, C], "sr": sr, "ms": round(ms, 4), "gbs": round(gbs, 1),
-                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "frac_hbm_nominal": round(gbs / NOMINAL_HBM_GBS, 4)})
+                         "frac_hbm": round(gbs / peaks["hbm_gbs"], 4), "frac_hbm_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+                         "hbm_roof_us": round(R * C * (2 + 0.5 + 1.0 / 32) / (peaks["hbm_gbs"] * 1e9) * 1e6, 2)})
         del x, out
+    x = torch.zeros((32, 32), dtype=torch.bfloat16, device=dev)
+    out = dict(codes=torch.empty((1, 32, 16), dtype=torch.uint8, device=dev),
+               scales=torch.empty((1, 32, 1), dtype=torch.uint8, device=dev))
+    floor = {"rn_us": round(1e3 * timed(x, out, False), 2), "sr_us": round(1e3 * timed(x, out, True), 2),
+             "what": "one 32x32 block (one CTA), same timing method: the cost of a launch with no data to move"}
     mxfp4.mxfp4_check_device_status()
-    return {"quant_sweep": rows, "l2": "flushed (256 MB write) before every timed launch", "iters": iters,
-            "warmup": warmup, "peak_source": peaks["source"] + " copy bandwidth"}
+    return {"quant_sweep": rows, "launch_floor": floor, "l2": "flushed (256 MB write) before every timed launch",
+            "iters": iters, "warmup": warmup, "peak_source": peaks["source"] + " copy bandwidth"}
 
 
 def run_reference(args):
@@ -617,12 +662,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-quant-sweep", action="store_true",
+                    help="skip the quantise-sweep leg after the step measurements")
     ap.add_argument("--quant-sweep", action="store_true",
                     help="time the 1x32 quantiser alone on the quantise-sweep shapes (L2 flushed) and exit")
     ap.add_argument("--oracle-timing", action="store_true",
                     help="print a fuller timing report of the CPU oracle (host only) and exit")
     ap.add_argument("--fused-steps", type=int, default=10,
-                    help="steps of the fused-epilogue variant timed after the main region (0: skip)")
+                    help="steps of each variant (binary32 / fused epilogue) timed interleaved after the main region "
+                         "(0: skip)")
     ap.add_argument("--experts", type=int, default=32,
                     help="smaller layers are for profiler captures only; the result line names the size")
     ap.add_argument("--tokens", type=int, default=16384)
@@ -646,6 +694,17 @@ def main():
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream()
+    gpu_uuid = None
+    try:
+        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        if not gpu_uuid.startswith("GPU-"):
+            gpu_uuid = "GPU-" + gpu_uuid
+    except Exception:
+        gpu_uuid = str(local)
+    # the clock sampler runs from before the warm-up steps, so the GPU does
+    # not sit idle (and drop its clocks) between the warm-up and the region
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
     for _ in range(args.warmup):
         layer.step()
     layer.mx.mxfp4_check_device_status()
@@ -654,16 +713,6 @@ def main():
     # per-kernel events over the timed steps
     evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
            for _ in range(args.steps)]
-    gpu_uuid = None
-    try:
-        gpu_uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        if not gpu_uuid.startswith("GPU-"):
-            gpu_uuid = "GPU-" + gpu_uuid
-    except Exception:
-        gpu_uuid = str(local)
-    clocks = ClockSampler(gpu_uuid)
-    clocks.start()
-    time.sleep(0.3)
     barrier(pg)
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -686,7 +735,11 @@ def main():
     gemm_ms = sum(per_kernel[k] for k in layer.gemm_flops)
     quant_ms = sum(per_kernel[k] for k in layer.quant_bytes)
     quant_gbs = sum(layer.quant_bytes.values()) / (quant_ms / 1e3) / 1e9
-    fp4_peak = peaks["bf16_sustained"] * NOMINAL_FP4_OVER_BF16
+    # kernels timed with events inside a sub-second region: the burst bf16
+    # peak (x 4, the datasheet's dense FP4:BF16 ratio) is the denominator
+    fp4_peak = peaks["bf16_burst"] * NOMINAL_FP4_OVER_BF16
+    fp4_sustained = peaks["bf16_sustained"] * NOMINAL_FP4_OVER_BF16
+    region_s = ms / 1e3
     dominant = max(per_kernel, key=lambda k: per_kernel[k])
     dom_ms = per_kernel[dominant]
     full_size = (args.experts, args.tokens) == (32, 16384)
@@ -695,8 +748,9 @@ def main():
         achieved = layer.gemm_flops[dominant] / (dom_ms / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak,
-                "peak_source": "%s sustained bf16 x %.0f (nominal FP4:BF16 dense ratio)" % (peaks["source"],
-                                                                                          NOMINAL_FP4_OVER_BF16),
+                "peak_source": "%s burst bf16 x %.0f (nominal FP4:BF16 dense ratio); the kernel is timed with CUDA "
+                               "events inside a %.2f s region" % (peaks["source"], NOMINAL_FP4_OVER_BF16, region_s),
+                "frac_sustained": achieved / fp4_sustained,
                 "kernel": dominant, "traffic": dom_traffic,
                 "hbm_frac": layer.gemm_out_bytes(dominant) / (dom_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
                 "peak_nominal": NOMINAL_FP4_TFLOPS, "frac_nominal": achieved / NOMINAL_FP4_TFLOPS}
@@ -717,40 +771,64 @@ def main():
         else:
             gbs = layer.quant_bytes[k] / (t / 1e3) / 1e9
             components[k] = {"ms": round(t, 4), "gbs": round(gbs, 1), "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    ck = clocks.summary(t0, t1)
 
-    # ---------------- fused-epilogue variant (side measurement, not the step above)
+    # ---------------- fused-epilogue variant, interleaved with the binary32 step
     # The same step with fprop/dgrad writing bf16 outputs plus their MXFP4
-    # quantisation straight from the accumulator instead of binary32.
+    # quantisation straight from the accumulator instead of binary32.  The
+    # two variants alternate step by step (the order flips every pair) in one
+    # region, each step synchronised so the clock samples taken during it are
+    # attributed to its variant.
     fused = None
     if args.fused_steps > 0:
         layer.alloc_fused()
+        clocks = ClockSampler(gpu_uuid)       # started before this section's warm-up steps
+        clocks.start()
         for _ in range(3):
+            layer.step()
             layer.step(fused=True)
         layer.mx.mxfp4_check_device_status()
-        fevs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
-                for _ in range(args.fused_steps)]
         torch.cuda.synchronize()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
+        res = {"binary32": {"win": [], "ms": [], "k": []}, "fused": {"win": [], "ms": [], "k": []}}
         for i in range(args.fused_steps):
-            layer.step(fevs[i], fused=True)
-        f1.record(stream)
-        torch.cuda.synchronize()
+            order = (("binary32", False), ("fused", True)) if i % 2 == 0 else (("fused", True), ("binary32", False))
+            for name, fz in order:
+                ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                w0 = time.time()
+                a0.record(stream)
+                layer.step(ev, fused=fz)
+                a1.record(stream)
+                torch.cuda.synchronize()
+                res[name]["win"].append((w0, time.time()))
+                res[name]["ms"].append(a0.elapsed_time(a1))
+                res[name]["k"].append({k: ev[k][0].elapsed_time(ev[k][1]) for k in layer.FUSED})
+        clocks.stop()
         layer.mx.mxfp4_check_device_status()
-        fk = {k: statistics.mean(e[k][0].elapsed_time(e[k][1]) for e in fevs) for k in layer.FUSED}
-        fused = {"steps": args.fused_steps, "ms_per_step": f0.elapsed_time(f1) / args.fused_steps,
-                 "kernels": {k: {"ms": round(fk[k], 4), "ms_binary32_out": round(per_kernel[k], 4),
-                                 "tflops": round(layer.gemm_flops[k] / (fk[k] / 1e3) / 1e12, 1),
-                                 "alg_gbs": round(layer.fused_out_bytes(k) / (fk[k] / 1e3) / 1e9, 1)}
-                             for k in layer.FUSED}}
+
+        def kmed(name, k):
+            return statistics.median(r[k] for r in res[name]["k"])
+        fused = {"steps_each": args.fused_steps, "interleaved": True,
+                 "ms_per_step": statistics.median(res["fused"]["ms"]),
+                 "ms_per_step_binary32": statistics.median(res["binary32"]["ms"]),
+                 "clocks_fused": clocks.summary_windows(res["fused"]["win"]),
+                 "clocks_binary32": clocks.summary_windows(res["binary32"]["win"]),
+                 "kernels": {k: {"ms": round(kmed("fused", k), 4), "ms_binary32_out": round(kmed("binary32", k), 4),
+                                 "tflops": round(layer.gemm_flops[k] / (kmed("fused", k) / 1e3) / 1e12, 1),
+                                 "alg_gbs": round(layer.fused_out_bytes(k) / (kmed("fused", k) / 1e3) / 1e9, 1)}
+                             for k in layer.FUSED},
+                 "what": "medians over steps; each step synchronised; per-step ms from CUDA events around the step"}
         del layer.fused_out
 
     # ---------------- end to end through the C ABI with host buffers
-    # Every step uploads its inputs from pinned host memory and reads its
-    # results back.  Two sets of device I/O buffers and three streams let the
-    # upload of step i+1, the step-i kernels and the download of step i-1 run
-    # at once (PCIe moves both directions concurrently).
-    io_in, io_out = ("x", "h", "dy_up", "dy_down"), ("dx", "dh")
+    # Every step uploads its inputs (X, H, dY_up, dY_down) from pinned host
+    # memory and reads every output of the step back (Y_up, Y_down, dX, dH,
+    # dW_up, dW_down).  The fp32 master weights and their de-oscillation
+    # state persist on the device between steps, as an optimizer keeps them.
+    # Two sets of device I/O buffers and three streams let the upload of step
+    # i+1, the step-i kernels and the download of step i-1 run at once (PCIe
+    # moves both directions concurrently).
+    io_in, io_out = ("x", "h", "dy_up", "dy_down"), ("y_up", "y_down", "dx", "dh", "dw_up", "dw_down")
     sets = [{n: getattr(layer, n) for n in io_in + io_out},
             {n: torch.empty_like(getattr(layer, n)) for n in io_in + io_out}]
     for n in io_in:
@@ -801,6 +879,39 @@ def main():
     e2e_value = step_flops * args.e2e_steps * world / (e2e_ms / 1e3) / 1e12
     for n in io_in + io_out:
         setattr(layer, n, sets[0][n])
+    del sets, host_in, host_out
+
+    # ---------------- quantise sweep (the 1x32 quantiser alone, L2 flushed)
+    # and the issue-rate (ALU) roof of the stochastic-rounding kernels
+    qs = None
+    if not args.no_quant_sweep:
+        qs = quant_sweep()
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = ck["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)
+    alu = {"sm_mhz": mhz, "issue": "%d SMs x %d schedulers x 1 warp instruction per cycle" % (n_sms, SMSP_PER_SM),
+           "kernels": {}}
+    for k, elems in (("dual_dy_up", layer.M * F), ("dual_dy_down", layer.M * D)):
+        ipe = SR_INST_PER_ELEMENT[k]
+        hbm_ms = layer.quant_bytes[k] / (peaks["hbm_gbs"] * 1e9) * 1e3
+        ent = {"elements": elems, "inst_per_element": ipe, "hbm_ms": round(hbm_ms, 4), "ms": round(per_kernel[k], 4)}
+        if ipe is not None:
+            alu_ms = issue_roof_ms(ipe, elems, n_sms, mhz)
+            ent.update(alu_ms=round(alu_ms, 4), roof_ms=round(max(alu_ms, hbm_ms), 4),
+                       frac_roof=round(max(alu_ms, hbm_ms) / per_kernel[k], 4))
+        alu["kernels"][k] = ent
+    if qs is not None:
+        for row in qs["quant_sweep"]:
+            if not row["sr"]:
+                continue
+            R, C = row["shape"]
+            ipe = SR_INST_PER_ELEMENT["rows_sr"]
+            hbm_ms = row["hbm_roof_us"] / 1e3
+            ent = {"elements": R * C, "inst_per_element": ipe, "hbm_ms": round(hbm_ms, 4), "ms": row["ms"]}
+            if ipe is not None:
+                alu_ms = issue_roof_ms(ipe, R * C, n_sms, mhz)
+                ent.update(alu_ms=round(alu_ms, 4), roof_ms=round(max(alu_ms, hbm_ms), 4),
+                           frac_roof=round(max(alu_ms, hbm_ms) / row["ms"], 4))
+            alu["kernels"]["quantise_sr_%dx%d" % (R, C)] = ent
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -810,7 +921,6 @@ def main():
                          % CPU_SAMPLE_ROWS +
                          "quantisations (2D de-oscillation W, SR dY, RHT-16 transposed operands); %.1f s on %d "
                          "threads of %d host cores" % (secs, threads, os.cpu_count() or 0)}
-    ck = clocks.summary(t0, t1)
     probe = fp4_mma_probe(layer.mx, stream)
     if roof["bound"] == "tensor":
         roof["peak_probe"] = probe
@@ -833,12 +943,16 @@ def main():
         "gemm_frac_fp4_probe": step_flops / (gemm_ms / 1e3) / 1e12 / probe,
         "roofline": roof, "components": components,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d_bytes),
-                "d2h_bytes_per_step": int(d2h_bytes)},
+                "d2h_bytes_per_step": int(d2h_bytes), "steps": args.e2e_steps,
+                "what": "inputs X, H, dY_up, dY_down uploaded and every output (Y_up, Y_down, dX, dH, dW_up, dW_down) "
+                        "read back each step; masters and de-oscillation state resident"},
         "gpu_launches": layer.launches_per_step * args.steps,
-        "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"], "reasons": ck["reasons"],
-                   "samples": ck["samples"]},
+        "clocks": {"sm_mhz": ck["sm_mhz"], "sm_max_mhz": ck["sm_max_mhz"], "sm_mhz_min": ck.get("sm_mhz_min"),
+                   "reasons": ck["reasons"], "samples": ck["samples"]},
         "cpu_baseline": cpu,
         "fused_epilogue": fused,
+        "quantise_sweep": qs,
+        "sr_alu_roof": alu,
     }
     if rank == 0:
         print(json.dumps(line))
