@@ -13,12 +13,18 @@
 //   - the leader CTA's single MMA thread issues tcgen05.mma.cta_group::2
 //     (M = 256, N = 192, K = 64) over both CTAs' shared memory and tensor
 //     memory, and its commits are multicast to both CTAs' barriers;
-//   - the UE8M0 scales are staged per CTA by four loader warps with
-//     tcgen05.st, in the layout of a 128 x 256 one-CTA MMA (every CTA holds its
+//   - warp 0 issues the operand boxes; warp 10 issues the UE8M0 scale copies
+//     into a ring of four slots of their own, so they run ahead of the
+//     operand ring;
+//   - four loader warps read a scale slot (and free it at once), wait until
+//     the stage's tensor-memory scale columns are free, and write them with
+//     tcgen05.st in the layout of a 128 x 256 one-CTA MMA (every CTA holds its
 //     own rows of A's scales and all of B's); the odd-tile offset of the
 //     192-wide B window is applied by the loaders, so a stage needs 40 scale
 //     columns and two 192-column accumulators still fit in TMEM.  The loaders
 //     arrive on the stage's full barrier, so the MMA thread waits once;
+//   - every role walks the cluster's units (group, m-tile pair, n-tile)
+//     with adds and bounded wraps, no division per unit;
 //   - four epilogue warps drain the accumulator: binary32 output in 8 KB TMA
 //     stores (two 32-column chunks through a [column block][row][32 floats]
 //     view of D), or with FUSED the bf16 output and its 1x32 MXFP4 codes;
@@ -46,7 +52,8 @@ constexpr int BK = 512;                          // elements per K-step (one bar
 constexpr int kSub = BK / 256;                   // 128-byte-wide swizzled boxes per operand and K-step
 constexpr int kChunks = BK / 128;                // 4-scale chunks per K-step
 constexpr int kStages = 3;
-constexpr int kThreads = 320;
+constexpr int kSfStages = 4;                     // scale ring: copies run ahead of the operand ring
+constexpr int kThreads = 352;
 constexpr uint32_t kABox = BM * 128;             // 16384: 128 rows x 256 elements
 constexpr uint32_t kBBox = BNH * 128;            // 12288:  96 rows x 256 elements
 constexpr uint32_t kABytes = kSub * kABox;
@@ -65,14 +72,14 @@ constexpr int kMaxGroups = 255;
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + kStages * kABytes;
 constexpr uint32_t kOffSFA = kOffB + kStages * kBBytes;
-constexpr uint32_t kOffSFB = kOffSFA + kStages * kSFABytes;
-constexpr uint32_t kOffEpi = kOffSFB + kStages * kSFBBytes;
+constexpr uint32_t kOffSFB = kOffSFA + kSfStages * kSFABytes;
+constexpr uint32_t kOffEpi = kOffSFB + kSfStages * kSFBBytes;
 constexpr uint32_t kOffBar = kOffEpi + 4 * 2 * kEpiBufBytes;
-constexpr uint32_t kNumBars = 3 * kStages + 2 + 2 + 1;  // full, empty, sffull, tfull, tempty, drain
+// full, empty (operand stages); sffull, sfempty (scale slots); tfull, tempty; drain
+constexpr uint32_t kNumBars = 2 * kStages + 2 * kSfStages + 2 + 2 + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kOffGroups = kOffMisc + 64;
-constexpr uint32_t kOffPrefix = kOffGroups + (kMaxGroups + 1) * 4;
-constexpr uint32_t kSmemBytes = kOffPrefix + (kMaxGroups + 1) * 4 + 1024;
+constexpr uint32_t kSmemBytes = kOffGroups + (kMaxGroups + 1) * 4 + 1024;
 static_assert(kOffB % 1024 == 0 && kOffEpi % 1024 == 0, "swizzled tiles must be 1024-aligned");
 static_assert(kABox % 1024 == 0 && kBBox % 1024 == 0, "boxes must hold whole swizzle atoms");
 static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
@@ -92,43 +99,68 @@ struct Unit {
     int64_t kbeg, kend;
 };
 
-// Units of work: (group, m-tile pair, n-tile).  Mode 0 pairs the 128-row
-// tiles inside each group (prefix[g] counts the units before group g); mode 1
-// pairs the row tiles of A (same for every group).
-__device__ __forceinline__ Unit unit_info(const Args& a, const int32_t* s_off, const int32_t* s_prefix, int64_t u) {
-    Unit un;
-    if (a.mode == 0) {
-        int lo = 0, hi = a.num_groups - 1;  // largest g with prefix[g] <= u
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_prefix[mid] <= u) lo = mid;
-            else hi = mid - 1;
-        }
-        const int64_t local = u - s_prefix[lo];
-        const int64_t p = local / a.n_tiles;
-        un.g = lo;
-        un.n0 = (local - p * a.n_tiles) * BN;
-        un.ma = s_off[lo] / BM + 2 * p;
-        un.mb = un.ma + 1;
-        un.vb = un.mb * BM < s_off[lo + 1];
-        un.kbeg = 0;
-        un.kend = a.K;
-    } else {
-        const int64_t pairs = (int64_t(a.m_tiles) + 1) / 2;
-        const int64_t per = pairs * a.n_tiles;
-        const int g = int(u / per);
-        const int64_t rem = u - int64_t(g) * per;
-        const int64_t p = rem / a.n_tiles;
-        un.g = g;
-        un.n0 = (rem - p * a.n_tiles) * BN;
-        un.ma = 2 * p;
-        un.mb = 2 * p + 1;
-        un.vb = un.mb < a.m_tiles;
-        un.kbeg = s_off[g];
-        un.kend = s_off[g + 1];
+// Units of work: (group, m-tile pair, n-tile), n-tile fastest.  Mode 0 pairs
+// the 128-row tiles inside each group (a group of t tiles has (t + 1) / 2
+// pairs); mode 1 pairs the row tiles of A, the same for every group, and the
+// groups split the contraction.  A cluster takes the units u = first,
+// first + step, ...; the walk advances (group g, pair p, n-tile n) by the
+// step with adds and bounded wraps -- a group's units are its pairs x
+// n_tiles, so the index carries from n into p and from p into the next group
+// with pairs (empty groups have none) -- with no division per unit.
+struct UnitWalk {
+    int g;
+    int32_t p, n, dp, dn;
+    __host__ __device__ static int32_t pairs_in(const Args& a, const int32_t* s_off, int g) {
+        return a.mode == 0 ? (((s_off[g + 1] - s_off[g]) / BM) + 1) / 2 : (a.m_tiles + 1) / 2;
     }
-    return un;
-}
+    __host__ __device__ void init(const Args& a, const int32_t* s_off, int64_t u, int64_t step) {
+        dp = int32_t(step / a.n_tiles);
+        dn = int32_t(step - int64_t(dp) * a.n_tiles);
+        int64_t local = u;
+        g = 0;
+        while (g < a.num_groups) {
+            const int64_t units = int64_t(pairs_in(a, s_off, g)) * a.n_tiles;
+            if (local < units) break;
+            local -= units;
+            ++g;
+        }
+        p = int32_t(local / a.n_tiles);
+        n = int32_t(local - int64_t(p) * a.n_tiles);
+    }
+    __host__ __device__ void advance(const Args& a, const int32_t* s_off) {
+        n += dn;
+        if (n >= a.n_tiles) {
+            n -= a.n_tiles;
+            ++p;
+        }
+        p += dp;
+        while (g < a.num_groups) {
+            const int32_t pg = pairs_in(a, s_off, g);
+            if (p < pg) break;
+            p -= pg;
+            ++g;
+        }
+    }
+    __host__ __device__ Unit unit(const Args& a, const int32_t* s_off) const {
+        Unit un;
+        un.g = g;
+        un.n0 = int64_t(n) * BN;
+        if (a.mode == 0) {
+            un.ma = s_off[g] / BM + 2 * int64_t(p);
+            un.mb = un.ma + 1;
+            un.vb = un.mb * BM < s_off[g + 1];
+            un.kbeg = 0;
+            un.kend = a.K;
+        } else {
+            un.ma = 2 * int64_t(p);
+            un.mb = un.ma + 1;
+            un.vb = un.mb < a.m_tiles;
+            un.kbeg = s_off[g];
+            un.kend = s_off[g + 1];
+        }
+        return un;
+    }
+};
 
 // FUSED (mode 0): the epilogue writes each output element as bf16 (round to
 // nearest even) and quantises every 32-column chunk of a row -- one lane's
@@ -149,15 +181,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // tensor memory (8 loader-warp arrivals); one wait per K-step
     uint64_t* full = bars;
     uint64_t* empty = bars + kStages;             // both: the pair's MMAs released the stage
-    uint64_t* sffull = bars + 2 * kStages;        // both: this CTA's scale chunks landed
-    uint64_t* tfull = bars + 3 * kStages;         // both: accumulator ready
-    uint64_t* tempty = bars + 3 * kStages + 2;    // leader: both CTAs drained the accumulator (8 warps)
-    uint64_t* drain = bars + 3 * kStages + 4;     // both: all of the pair's MMAs completed
+    uint64_t* sffull = bars + 2 * kStages;        // both: a scale slot's chunks landed
+    uint64_t* sfempty = sffull + kSfStages;       // both: the 4 loader warps have read a scale slot
+    uint64_t* tfull = sfempty + kSfStages;        // both: accumulator ready
+    uint64_t* tempty = tfull + 2;                 // leader: both CTAs drained the accumulator (8 warps)
+    uint64_t* drain = tempty + 2;                 // both: all of the pair's MMAs completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
     volatile int* offsets_ok = reinterpret_cast<volatile int*>(smem + kOffMisc + 16);
+    int64_t* s_total = reinterpret_cast<int64_t*>(smem + kOffMisc + 24);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + kOffGroups);
-    int32_t* s_prefix = reinterpret_cast<int32_t*>(smem + kOffPrefix);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
@@ -169,7 +202,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 2 + 8);
             mbar_init(&empty[s], 1);
+        }
+        for (int s = 0; s < kSfStages; ++s) {
             mbar_init(&sffull[s], 1);
+            mbar_init(&sfempty[s], 4);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
@@ -197,24 +233,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const bool v = gemm::offsets_valid(a, s_off);
         *offsets_ok = v ? 1 : 0;
         if (!v && blockIdx.x == 0) atomicOr(a.status, kStatusBadInput);
-        if (a.mode == 0) {
-            int32_t acc = 0;
-            for (int g = 0; g < a.num_groups; ++g) {
-                s_prefix[g] = acc;
-                const int32_t t = v ? (s_off[g + 1] - s_off[g]) / BM : 0;
-                acc += ((t + 1) / 2) * a.n_tiles;
-            }
-            s_prefix[a.num_groups] = acc;
-        }
+        int64_t units = 0;
+        if (v)
+            for (int g = 0; g < a.num_groups; ++g) units += int64_t(UnitWalk::pairs_in(a, s_off, g)) * a.n_tiles;
+        *s_total = units;
     }
     __syncthreads();
     cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated before any cross-CTA traffic
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    int64_t total = 0;
-    if (*offsets_ok)
-        total = a.mode == 0 ? int64_t(s_prefix[a.num_groups])
-                            : int64_t(a.num_groups) * ((int64_t(a.m_tiles) + 1) / 2) * a.n_tiles;
+    const int64_t total = *s_total;   // 0 when the offsets were rejected
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -227,20 +255,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 pend_phase[s] = 0;
             }
             bool ok = true;
-            for (int64_t u = cluster; u < total && ok; u += nclusters) {
-                const Unit un = unit_info(a, s_off, s_prefix, u);
+            UnitWalk uw;
+            uw.init(a, s_off, cluster, nclusters);
+            for (int64_t u = cluster; u < total && ok; u += nclusters, uw.advance(a, s_off)) {
+                const Unit un = uw.unit(a, s_off);
                 const int64_t mt = (leader || !un.vb) ? un.ma : un.mb;   // an idle half reloads ma (never stored)
-                const int64_t rbb = un.n0 / 128;
-                const bool has_rb1 = rbb + 1 < a.nrb_b;
-                const uint8_t* sfb_g = a.sfb + (a.mode == 0 ? int64_t(un.g) * a.sfb_group_bytes : 0);
                 for (int64_t k = un.kbeg; k < un.kend; k += BK) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.status, kRoleProducer)) {
                         ok = false;
                         break;
                     }
-                    const int64_t chunk = k >> 7;
-                    const uint32_t nca = uint32_t(imin64(kChunks, a.nchunk_a - chunk));
-                    const uint32_t ncb = uint32_t(imin64(kChunks, a.nchunk_b - chunk));
                     const int nsub = un.kend - k > 256 ? 2 : 1;   // boxes of 256 elements this K-step needs
                     const uint32_t full_c = mapa_shared(smem_u32(&full[stage]), 0);
                     mbar_arrive_expect_tx_cluster(full_c, uint32_t(nsub) * (kABox + kBBox));
@@ -267,17 +291,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 tma_load_2d_pair(sB + j * kBBox, &tmB, full_c, xk, brow);
                         }
                     }
-                    // then the scales: small, they reach tensor memory (bulk copy,
-                    // loader warps) well before the operand tiles land, so the
-                    // operand copies go first
-                    mbar_arrive_expect_tx(&sffull[stage], nca * 512u + ncb * 512u * (has_rb1 ? 2u : 1u));
-                    bulk_load(smem + kOffSFA + stage * kSFABytes, a.sfa + (mt * a.nchunk_a + chunk) * 512, nca * 512u,
-                              &sffull[stage]);
-                    bulk_load(smem + kOffSFB + stage * kSFBBytes, sfb_g + (rbb * a.nchunk_b + chunk) * 512,
-                              ncb * 512u, &sffull[stage]);
-                    if (has_rb1)
-                        bulk_load(smem + kOffSFB + stage * kSFBBytes + kChunks * 512,
-                                  sfb_g + ((rbb + 1) * a.nchunk_b + chunk) * 512, ncb * 512u, &sffull[stage]);
                     pend[stage] = true;
                     pend_phase[stage] = phase;
                     if (++stage == kStages) {
@@ -286,25 +299,77 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            // drain: this CTA's scale copies (local barrier); the leader also
-            // waits for the operand tiles of both CTAs (they complete on its
-            // `full` barriers)
+            // drain: the leader waits for the operand tiles of both CTAs (they
+            // complete on its `full` barriers)
             for (int s = 0; s < kStages; ++s) {
-                if (!pend[s]) continue;
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(&sffull[s], pend_phase[s])) {
-                    if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+                if (!pend[s] || !leader) continue;
+                const uint64_t t1 = globaltimer_ns();
+                while (!mbar_try_wait(&full[s], pend_phase[s])) {
+                    if (globaltimer_ns() - t1 > kWaitBudgetNs) {
                         atomicOr(a.status, kStatusTimeout | kRoleTeardown);
                         break;
                     }
                 }
-                if (leader) {
-                    const uint64_t t1 = globaltimer_ns();
-                    while (!mbar_try_wait(&full[s], pend_phase[s])) {
-                        if (globaltimer_ns() - t1 > kWaitBudgetNs) {
-                            atomicOr(a.status, kStatusTimeout | kRoleTeardown);
-                            break;
-                        }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ scale copies (both CTAs)
+        // The UE8M0 scales of each K-step go into a ring of kSfStages slots of
+        // their own, freed as soon as the loader warps have read them, so the
+        // copies run ahead of the operand ring and the scales are in registers
+        // by the time a stage's tensor-memory columns are free.
+        if (lane == 0) {
+            uint32_t slot = 0, sphase = 0;
+            bool pend[kSfStages];
+            uint32_t pend_phase[kSfStages];
+            for (int i = 0; i < kSfStages; ++i) {
+                pend[i] = false;
+                pend_phase[i] = 0;
+            }
+            bool ok = true;
+            UnitWalk uw;
+            uw.init(a, s_off, cluster, nclusters);
+            for (int64_t u = cluster; u < total && ok; u += nclusters, uw.advance(a, s_off)) {
+                const Unit un = uw.unit(a, s_off);
+                const int64_t mt = (leader || !un.vb) ? un.ma : un.mb;
+                const int64_t rbb = un.n0 / 128;
+                const bool has_rb1 = rbb + 1 < a.nrb_b;
+                const uint8_t* sfb_g = a.sfb + (a.mode == 0 ? int64_t(un.g) * a.sfb_group_bytes : 0);
+                for (int64_t k = un.kbeg; k < un.kend; k += BK) {
+                    if (!mbar_wait_bounded(&sfempty[slot], sphase ^ 1u, abort_flag, a.status, kRoleScales)) {
+                        ok = false;
+                        break;
+                    }
+                    const int64_t chunk = k >> 7;
+                    const uint32_t nca = uint32_t(imin64(kChunks, a.nchunk_a - chunk));
+                    const uint32_t ncb = uint32_t(imin64(kChunks, a.nchunk_b - chunk));
+                    mbar_arrive_expect_tx(&sffull[slot], nca * 512u + ncb * 512u * (has_rb1 ? 2u : 1u));
+                    bulk_load(smem + kOffSFA + slot * kSFABytes, a.sfa + (mt * a.nchunk_a + chunk) * 512, nca * 512u,
+                              &sffull[slot]);
+                    bulk_load(smem + kOffSFB + slot * kSFBBytes, sfb_g + (rbb * a.nchunk_b + chunk) * 512,
+                              ncb * 512u, &sffull[slot]);
+                    if (has_rb1)
+                        bulk_load(smem + kOffSFB + slot * kSFBBytes + kChunks * 512,
+                                  sfb_g + ((rbb + 1) * a.nchunk_b + chunk) * 512, ncb * 512u, &sffull[slot]);
+                    pend[slot] = true;
+                    pend_phase[slot] = sphase;
+                    if (++slot == kSfStages) {
+                        slot = 0;
+                        sphase ^= 1u;
+                    }
+                }
+            }
+            // drain: every copy this thread issued has landed before the CTA
+            // may exit (the loaders consume every slot on a normal exit; after
+            // an abort some may still be in flight)
+            for (int i = 0; i < kSfStages; ++i) {
+                if (!pend[i]) continue;
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(&sffull[i], pend_phase[i])) {
+                    if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+                        atomicOr(a.status, kStatusTimeout | kRoleTeardown);
+                        break;
                     }
                 }
             }
@@ -317,8 +382,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 uint32_t stage = 0, phase = 0;
                 uint32_t acc = 0, acc_phase = 0;
                 bool ok = true;
-                for (int64_t u = cluster; u < total && ok; u += nclusters) {
-                    const Unit un = unit_info(a, s_off, s_prefix, u);
+                UnitWalk uw;
+                uw.init(a, s_off, cluster, nclusters);
+                for (int64_t u = cluster; u < total && ok; u += nclusters, uw.advance(a, s_off)) {
+                    const Unit un = uw.unit(a, s_off);
                     if (un.kend <= un.kbeg) continue;
                     if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, abort_flag, a.status, kRoleMma)) {
                         ok = false;
@@ -366,20 +433,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale loaders (both CTAs)
+        // Per K-step: read the scale slot into registers and free it, wait
+        // until the pair's MMAs of the stage's previous round have completed
+        // (its tensor-memory scale columns are then free), write them, and
+        // arrive on the leader's `full` barrier of the stage.
         const int q = warp & 3;
-        uint32_t stage = 0, phase = 0;
+        uint32_t stage = 0, phase = 0;     // operand / tensor-memory stage
+        uint32_t slot = 0, sphase = 0;     // scale slot
         bool ok = true;
-        for (int64_t u = cluster; u < total && ok; u += nclusters) {
-            const Unit un = unit_info(a, s_off, s_prefix, u);
+        UnitWalk uw;
+        uw.init(a, s_off, cluster, nclusters);
+        for (int64_t u = cluster; u < total && ok; u += nclusters, uw.advance(a, s_off)) {
+            const Unit un = uw.unit(a, s_off);
             const int shift = int((un.n0 & 127) >> 5);   // 0 or 2: the 192-wide window inside 256 rows of B
             for (int64_t k = un.kbeg; k < un.kend; k += BK) {
-                const bool got = mbar_wait_bounded(&sffull[stage], phase, abort_flag, a.status, kRoleScales);
+                const bool got = mbar_wait_bounded(&sffull[slot], sphase, abort_flag, a.status, kRoleScales);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* sfa_s = smem + kOffSFA + stage * kSFABytes + lane * 16;
-                const uint8_t* sfb_s = smem + kOffSFB + stage * kSFBBytes + lane * 16;
+                const uint8_t* sfa_s = smem + kOffSFA + slot * kSFABytes + lane * 16;
+                const uint8_t* sfb_s = smem + kOffSFB + slot * kSFBBytes + lane * 16;
                 uint32_t ra[16], rb[24];
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
@@ -391,6 +465,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < 6; ++j) rb[6 * c + j] = shift ? w8[j + 2] : w8[j];
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfempty[slot]);
+                if (++slot == kSfStages) {
+                    slot = 0;
+                    sphase ^= 1u;
+                }
+                const bool free_cols = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, a.status, kRoleScales);
+                if (!__all_sync(0xFFFFFFFFu, free_cols)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();   // the tensor-memory writes follow the MMAs that read these columns
                 const uint32_t sf_cols = tmem_base + (uint32_t(32 * q) << 16) + kSfCol0 + stage * kSfColsPerStage;
                 tmem_st_32x32b_x16(sf_cols, ra);
                 uint32_t rb_lo[16], rb_hi[8];
@@ -419,8 +505,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         uint32_t acc = 0, acc_phase = 0;
         uint32_t buf = 0;
         bool ok = true;
-        for (int64_t u = cluster; u < total && ok; u += nclusters) {
-            const Unit un = unit_info(a, s_off, s_prefix, u);
+        UnitWalk uw;
+        uw.init(a, s_off, cluster, nclusters);
+        for (int64_t u = cluster; u < total && ok; u += nclusters, uw.advance(a, s_off)) {
+            const Unit un = uw.unit(a, s_off);
             const bool zero = un.kend <= un.kbeg;
             const bool valid = leader || un.vb;
             const int64_t mt = leader ? un.ma : un.mb;
