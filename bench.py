@@ -396,7 +396,7 @@ class ClockSampler:
         for r in rows:
             reasons |= r[3]
         return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max(r[2] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows)}
+                "sm_mhz_min": min(r[1] for r in rows), "reasons": sorted(reasons), "samples": len(rows)}
 
 
 # ---------------------------------------------------------------------------
@@ -556,7 +556,8 @@ def quant_sweep(iters=20, warmup=3, stream=None):
     (bf16 Gaussian draws on the device -- the kernels' time does not depend
     on the values --, RHT-16, nearest and stochastic rounding):
     median of `iters` CUDA-event timings after `warmup`, with L2 flushed
-    (a 256 MB write) before every timed launch.  Bytes per element: 2 in,
+    (a 256 MB write) before every timed launch and the GPU held by a short
+    spin until the launch is queued.  Bytes per element: 2 in,
     1/2 + 1/32 out.  The launch floor is the same measurement on a single
     32 x 32 block (one CTA): what a launch costs with no data to move."""
     import numpy as np
@@ -571,6 +572,10 @@ def quant_sweep(iters=20, warmup=3, stream=None):
         ts = []
         for i in range(warmup + iters):
             flush.zero_()
+            # hold the GPU (a spin of ~0.1 ms) so the launch and both events
+            # are queued before the GPU reaches the first event: the interval
+            # then holds the kernel alone, not the host's time to launch it
+            torch.cuda._sleep(200000)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             mxfp4.quantize(x, rht_seed=1, sr_seed=1 if sr else None, sr_offset=i, scales=True, out=out)
@@ -795,6 +800,9 @@ def main():
             for name, fz in order:
                 ev = {k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in KERNELS}
                 a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                # a spin of ~1 ms holds the GPU until the whole step is queued,
+                # so the host's launch time stays out of the step's interval
+                torch.cuda._sleep(2000000)
                 w0 = time.time()
                 a0.record(stream)
                 layer.step(ev, fused=fz)

@@ -275,3 +275,17 @@ def test_tensor_core_scale_layout_is_a_bijection(libpath):
         assert len(np.unique(off)) == R * S
         if R % 128 == 0 and S % 4 == 0:
             assert R * S == size
+
+
+def test_pair_gemm_unit_walk_matches_direct_decomposition(tmp_path):
+    """The pair GEMM's division-free unit walk visits, for every cluster,
+    exactly the units of the direct decomposition of u = cluster, cluster +
+    step, ... (random expert layouts with empty experts, both modes); checked
+    by a host program built from the kernel's own header."""
+    src = os.path.join(ROOT, "tests", "native", "unit_walk_check.cu")
+    exe = str(tmp_path / "unit_walk_check")
+    subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I",
+                    os.path.join(ROOT, "fp4_precision_numerics_b200", "csrc"), "-I", os.path.join(ROOT, "include"),
+                    "-o", exe, src, "-lcuda"], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    assert out.startswith("ok") and int(out.split()[1]) > 10 ** 6, out
