@@ -266,15 +266,21 @@ class Layer:
 # DRAM bytes per launch on the full workload (32 experts, 16384 tokens):
 # ncu dram__bytes_read.sum + dram__bytes_write.sum of each launch of the
 # 8-expert / 4096-token layer, whose every tensor is exactly a quarter of the
-# full one, times 4.  An entry must go back to None when its kernel changes.
+# full one, times 4; one kernel and at most three launches per capture (the
+# commands are in profiles/moe_layer_small_dram_counters.md).  An entry must
+# go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
     "deosc_up": 4 * (664.6e6 + 240.8e6), "deosc_down": 4 * (332.3e6 + 103.6e6),
     "dual_x": 4 * (97.4e6 + 18.0e6), "dual_h": 4 * (97.4e6 + 16.1e6),
     "dual_dy_up": 4 * (194.7e6 + 67.2e6), "dual_dy_down": 4 * (97.4e6 + 16.1e6),
-    "fprop_up": 4 * (97.0e6 + 333.7e6), "fprop_down": 4 * (61.3e6 + 139.5e6),
-    "dgrad_up": 4 * (122.6e6 + 153.2e6), "dgrad_down": 4 * (61.3e6 + 139.4e6),
-    "wgrad_up": 4 * (78.7e6 + 473.1e6), "wgrad_down": 4 * (51.9e6 + 206.7e6),
+    "fprop_up": 4 * (97.13e6 + 332.59e6), "fprop_down": 4 * (61.32e6 + 135.22e6),
+    "dgrad_up": 4 * (122.53e6 + 149.11e6), "dgrad_down": 4 * (61.32e6 + 137.45e6),
+    "wgrad_up": 4 * (78.72e6 + 467.04e6), "wgrad_down": 4 * (51.96e6 + 202.02e6),
 }
+
+KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
+           "dual_dy_down", "dgrad_down", "wgrad_up", "wgrad_down"]
+
 
 # Thread instructions per element of the stochastic-rounding quantisers:
 # ncu smsp__inst_executed.sum x 32 / elements of one launch (profiles/ gives
@@ -290,9 +296,6 @@ def issue_roof_ms(inst_per_element, elements, n_sms, sm_mhz):
     warp_inst = inst_per_element * elements / 32.0
     return warp_inst / (n_sms * SMSP_PER_SM) / (sm_mhz * 1e6) * 1e3
 
-
-KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
-           "dual_dy_down", "dgrad_down", "wgrad_up", "wgrad_down"]
 
 
 # ---------------------------------------------------------------------------
