@@ -270,9 +270,9 @@ class Layer:
 # commands are in profiles/moe_layer_small_dram_counters.md).  An entry must
 # go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": 4 * (664.6e6 + 240.8e6), "deosc_down": 4 * (332.3e6 + 103.6e6),
-    "dual_x": 4 * (97.4e6 + 18.0e6), "dual_h": 4 * (97.4e6 + 16.1e6),
-    "dual_dy_up": 4 * (194.7e6 + 67.2e6), "dual_dy_down": 4 * (97.4e6 + 16.1e6),
+    "deosc_up": 4 * (664.46e6 + 240.09e6), "deosc_down": 4 * (332.40e6 + 99.58e6),
+    "dual_x": 4 * (97.43e6 + 15.15e6), "dual_h": 4 * (97.42e6 + 12.05e6),
+    "dual_dy_up": 4 * (194.73e6 + 67.89e6), "dual_dy_down": 4 * (97.43e6 + 11.64e6),
     "fprop_up": 4 * (97.13e6 + 332.59e6), "fprop_down": 4 * (61.32e6 + 135.22e6),
     "dgrad_up": 4 * (122.53e6 + 149.11e6), "dgrad_down": 4 * (61.32e6 + 137.45e6),
     "wgrad_up": 4 * (78.72e6 + 467.04e6), "wgrad_down": 4 * (51.96e6 + 202.02e6),
