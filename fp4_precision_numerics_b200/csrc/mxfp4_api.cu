@@ -174,12 +174,23 @@ mxfp4_status launch_rows(const mxfp4::QuantArgs& qa, bool rht, bool sr, cudaStre
     if (qa.groups * qa.rows >= (int64_t(1) << 31))
         return fail(MXFP4_ERR_UNSUPPORTED_SHAPE, "mxfp4_quantize: groups * rows must be < 2^31");
     const int64_t work = qa.groups * qa.rows * (qa.cols / 32);
-    const unsigned grid = grid_for(work, 256);
-    if (rht && sr) mxfp4::quant1d_rows_kernel<InT, true, true><<<grid, 256, 0, st>>>(qa);
-    else if (rht) mxfp4::quant1d_rows_kernel<InT, true, false><<<grid, 256, 0, st>>>(qa);
-    else if (sr) mxfp4::quant1d_rows_kernel<InT, false, true><<<grid, 256, 0, st>>>(qa);
-    else mxfp4::quant1d_rows_kernel<InT, false, false><<<grid, 256, 0, st>>>(qa);
-    return check_launch("mxfp4_quantize(1d)");
+    // Grid: a tensor of at most 16 CTAs of work per resident CTA slot runs as
+    // one grid-stride pass of exactly the resident CTAs (no last wave of
+    // CTAs to wait for: 4096 x 2880 and 16384 x 2880 ran 8-10% faster); a
+    // larger one keeps 16 CTAs per SM, which the block scheduler backfills
+    // (65536 x 5760 with SR ran 5% slower as one resident pass).
+    auto go = [&](auto kern) -> mxfp4_status {
+        const int64_t blocks = (work + 255) / 256;
+        const int64_t resident = resident_ctas(kern, 256, 0);
+        const int64_t cap = blocks <= 16 * resident ? resident : int64_t(num_sms()) * 16;
+        const unsigned grid = unsigned(blocks < 1 ? 1 : (blocks < cap ? blocks : cap));
+        kern<<<grid, 256, 0, st>>>(qa);
+        return check_launch("mxfp4_quantize(1d)");
+    };
+    if (rht && sr) return go(mxfp4::quant1d_rows_kernel<InT, true, true>);
+    if (rht) return go(mxfp4::quant1d_rows_kernel<InT, true, false>);
+    if (sr) return go(mxfp4::quant1d_rows_kernel<InT, false, true>);
+    return go(mxfp4::quant1d_rows_kernel<InT, false, false>);
 }
 
 bool make_map_plain(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
