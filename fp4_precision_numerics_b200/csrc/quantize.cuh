@@ -700,7 +700,7 @@ __device__ __forceinline__ void quant2d_block(const QuantArgs& a, int64_t g, int
 }
 
 constexpr int kQ2dWarps = 8;   // warps (blocks) per CTA
-constexpr int kCoalBlkRows = 1, kCoalBlkCols = 8;   // the coalesced kernel's CTA: 1 x 8 blocks
+constexpr int kCoalBlkRows = 8, kCoalBlkCols = 1;   // the coalesced kernel's CTA: a column of 8 blocks
 constexpr int kCoalWarps = kCoalBlkRows * kCoalBlkCols;   // one warp per block
 
 template <typename InT, bool RHT, bool SR, bool DEOSC>
@@ -830,27 +830,16 @@ __device__ __forceinline__ void nib_swap(uint32_t (&w)[4]) {
     }
 }
 
+// One 32x32 block of the coalesced layout (lane 8q + c holds rows 4k + q,
+// elements 4c..4c+3): block maximum, scale, codes, de-oscillation state,
+// and the block's W^T codes, which go to *ct (16 bytes of W^T row
+// c0 + 4c + q) for the CTA to write out.
 template <typename InT, bool DEOSC>
-__global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __grid_constant__ QuantArgs a) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__device__ __forceinline__ void coal_block(const QuantArgs& a, int64_t g, int64_t bi, int64_t bj, int lane,
+                                           uint4* ct) {
     const int q = lane >> 3, c = lane & 7;
     const int64_t R = a.rows, C = a.cols;
     const int64_t nbr = R >> 5, nbc = C >> 5;
-    // A CTA takes a tile of kCoalBlkRows x kCoalBlkCols neighbouring blocks
-    // aligned to the block grid, so the row segments it reads and writes
-    // start on tile boundaries and are not shared with another CTA (a
-    // straight run of 8 blocks along a block row that wraps at the row end
-    // left CTAs sharing partly written lines).
-    const uint32_t tiles_c = uint32_t((nbc + kCoalBlkCols - 1) / kCoalBlkCols);
-    const uint32_t tiles_r = uint32_t((nbr + kCoalBlkRows - 1) / kCoalBlkRows);
-    const uint32_t per_g = tiles_r * tiles_c;
-    const uint32_t cta = blockIdx.x;
-    const int64_t g = cta / per_g;
-    const uint32_t rem = cta - uint32_t(g) * per_g;
-    const uint32_t ti = rem / tiles_c, tj = rem - ti * tiles_c;
-    const int64_t bi = int64_t(ti) * kCoalBlkRows + warp / kCoalBlkCols;
-    const int64_t bj = int64_t(tj) * kCoalBlkCols + warp % kCoalBlkCols;
-    if (g >= a.groups || bi >= nbr || bj >= nbc) return;
     const int64_t c0 = bj * 32;
     const InT* in = static_cast<const InT*>(a.in) + g * R * a.ld;
     const int64_t row0 = g * R + bi * 32;   // global row of the block's row 0
@@ -959,11 +948,48 @@ __global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __g
         nib_swap<1, 4>(w);
         nib_swap<2, 3>(w);
         nib_swap<3, 4>(w);
-        const int64_t tr = g * C + c0 + 4 * c + q;   // row of W^T
-        *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + bi * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *ct = make_uint4(w[0], w[1], w[2], w[3]);   // W^T row c0 + 4c + q, bytes 16 bi .. 16 bi + 15
         if (a.scales_mma_t)
             a.scales_mma_t[g * mma_scale_bytes(C, nbr) + mma_scale_offset(c0 + lane, bi, nbr)] = uint8_t(sb);
     }
+}
+
+
+// A CTA takes a grid-aligned column of kCoalBlkRows blocks, one warp each.
+// Their W^T codes are 16-byte pieces of the same 32 W^T rows at consecutive
+// offsets, so they are staged in shared memory and written as whole
+// 128-byte row segments (a 16-byte piece per lane per block leaves half
+// sectors scattered over 32 rows and made the W^T stores the launch's
+// costliest part).  The masters are read in 128-byte row segments.
+template <typename InT, bool DEOSC>
+__global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __grid_constant__ QuantArgs a) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t R = a.rows, C = a.cols;
+    const int64_t nbr = R >> 5, nbc = C >> 5;
+    const uint32_t tiles_c = uint32_t((nbc + kCoalBlkCols - 1) / kCoalBlkCols);
+    const uint32_t tiles_r = uint32_t((nbr + kCoalBlkRows - 1) / kCoalBlkRows);
+    const uint32_t per_g = tiles_r * tiles_c;
+    const uint32_t cta = blockIdx.x;
+    const int64_t g = cta / per_g;
+    const uint32_t rem = cta - uint32_t(g) * per_g;
+    const uint32_t ti = rem / tiles_c, tj = rem - ti * tiles_c;
+    const int bil = warp / kCoalBlkCols, bjl = warp % kCoalBlkCols;
+    const int64_t bi = int64_t(ti) * kCoalBlkRows + bil;
+    const int64_t bj = int64_t(tj) * kCoalBlkCols + bjl;
+    __shared__ uint4 s_ct[kCoalBlkCols][32][kCoalBlkRows];   // W^T pieces: [block column][lane][block row]
+    if (g < a.groups && bi < nbr && bj < nbc) coal_block<InT, DEOSC>(a, g, bi, bj, lane, &s_ct[bjl][lane][bil]);
+    if (!a.codes_t || g >= a.groups) return;   // uniform over the CTA
+    __syncthreads();
+    // thread t writes piece t % kCoalBlkRows of W^T row t / kCoalBlkRows, so
+    // each warp's store covers whole row segments
+    static_assert(kCoalBlkCols * 32 * kCoalBlkRows == kCoalWarps * 32, "one W^T piece per thread");
+    const int p = int(threadIdx.x) % kCoalBlkRows, pr = int(threadIdx.x) / kCoalBlkRows;
+    const int wb = pr >> 5, l = pr & 31;
+    const int64_t bis = int64_t(ti) * kCoalBlkRows + p;
+    const int64_t bjs = int64_t(tj) * kCoalBlkCols + wb;
+    if (bis >= nbr || bjs >= nbc) return;
+    const int64_t tr = g * C + bjs * 32 + 4 * (l & 7) + (l >> 3);   // row of W^T
+    *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + bis * 16) = s_ct[wb][l][p];
 }
 
 // ---------------------------------------------------------------------------
