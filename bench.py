@@ -270,7 +270,7 @@ class Layer:
 # commands are in profiles/moe_layer_small_dram_counters.md).  An entry must
 # go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": 4 * (664.46e6 + 240.09e6), "deosc_down": 4 * (332.40e6 + 99.58e6),
+    "deosc_up": 4 * (663.90e6 + 243.15e6), "deosc_down": None,   # deosc_down: not yet captured with the column-of-8 kernel
     "dual_x": 4 * (97.43e6 + 15.15e6), "dual_h": 4 * (97.42e6 + 12.05e6),
     "dual_dy_up": 4 * (194.73e6 + 67.89e6), "dual_dy_down": 4 * (97.43e6 + 11.64e6),
     "fprop_up": 4 * (97.13e6 + 332.59e6), "fprop_down": 4 * (61.32e6 + 135.22e6),
