@@ -253,8 +253,10 @@ def test_rht_non_finite_and_overflow(axis):
 
 # ----------------------------------------------------------- de-oscillation
 @pytest.mark.parametrize("freeze_lower", [False, True])
-def test_deosc_steps_bit_exact(freeze_lower):
-    G, R, C = 2, 256, 512
+@pytest.mark.parametrize("shape", [(2, 256, 512), (3, 160, 96)])
+def test_deosc_steps_bit_exact(freeze_lower, shape):
+    # (3, 160, 96): 5 block rows, so the kernel's last column of 8 blocks is ragged
+    G, R, C = shape
     w = synth.deosc_master(groups=G, rows=R, cols=C, seed=5)
     st_ref = np.zeros((G, R, C), dtype=np.uint8)
     wd = dev_f32(w)
