@@ -278,6 +278,31 @@ DRAM_BYTES_FULL = {
     "wgrad_up": 4 * (78.72e6 + 467.04e6), "wgrad_down": 4 * (51.96e6 + 202.02e6),
 }
 
+def gemm_roofline(flops, alg_bytes, ms, fp4_peak, fp4_sustained, hbm_gbs, tensor_src, hbm_src):
+    """Roofline entry of one GEMM launch.  The kernel is bound by whichever
+    roof takes longer for its algorithmic work: its flops at the FP4 peak
+    (TFLOP/s), or its bytes (operand codes and scales once, the binary32
+    output once) at the HBM peak (GB/s).  That roof gives `bound`, `achieved`,
+    `peak` and `frac`; the fractions against the other roof are kept beside
+    them."""
+    tflops = flops / (ms / 1e3) / 1e12
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    t_tensor_ms = flops / (fp4_peak * 1e12) * 1e3
+    t_hbm_ms = alg_bytes / (hbm_gbs * 1e9) * 1e3
+    if t_hbm_ms > t_tensor_ms:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                "peak_source": hbm_src, "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": gbs / NOMINAL_HBM_GBS}
+    else:
+        roof = {"bound": "tensor", "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s", "frac": tflops / fp4_peak,
+                "peak_source": tensor_src, "peak_nominal": NOMINAL_FP4_TFLOPS,
+                "frac_nominal": tflops / NOMINAL_FP4_TFLOPS}
+    roof.update({"alg_bytes": alg_bytes, "roof_ms": {"tensor": round(t_tensor_ms, 4), "hbm": round(t_hbm_ms, 4)},
+                 "tflops": tflops, "frac_tensor": tflops / fp4_peak, "peak_tensor": fp4_peak,
+                 "peak_tensor_source": tensor_src, "frac_tensor_sustained": tflops / fp4_sustained,
+                 "frac_tensor_nominal": tflops / NOMINAL_FP4_TFLOPS, "gbs": gbs, "frac_hbm": gbs / hbm_gbs})
+    return roof
+
+
 KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down", "dual_dy_up", "dgrad_up",
            "dual_dy_down", "dgrad_down", "wgrad_up", "wgrad_down"]
 
@@ -753,30 +778,11 @@ def main():
     full_size = (args.experts, args.tokens) == (32, 16384)
     dom_traffic = DRAM_BYTES_FULL.get(dominant) if full_size else None
     if dominant in layer.gemm_flops:
-        # a GEMM is bound by whichever roof takes longer for its algorithmic
-        # work: its flops at the FP4 peak, or its bytes (operands once, the
-        # binary32 output once) at the HBM peak; both fractions are reported
-        tflops = layer.gemm_flops[dominant] / (dom_ms / 1e3) / 1e12
-        alg_bytes = layer.gemm_out_bytes(dominant)
-        gbs = alg_bytes / (dom_ms / 1e3) / 1e9
-        t_tensor_ms = layer.gemm_flops[dominant] / (fp4_peak * 1e12) * 1e3
-        t_hbm_ms = alg_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
         tensor_src = ("%s burst bf16 x %.0f (nominal FP4:BF16 dense ratio); the kernel is timed with CUDA events "
                       "inside a %.2f s region" % (peaks["source"], NOMINAL_FP4_OVER_BF16, region_s))
-        if t_hbm_ms > t_tensor_ms:
-            roof = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                    "peak_nominal": NOMINAL_HBM_GBS, "frac_nominal": gbs / NOMINAL_HBM_GBS}
-        else:
-            roof = {"bound": "tensor", "achieved": tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                    "frac": tflops / fp4_peak, "peak_source": tensor_src,
-                    "peak_nominal": NOMINAL_FP4_TFLOPS, "frac_nominal": tflops / NOMINAL_FP4_TFLOPS}
-        roof.update({"kernel": dominant, "traffic": dom_traffic, "alg_bytes": alg_bytes,
-                     "roof_ms": {"tensor": round(t_tensor_ms, 4), "hbm": round(t_hbm_ms, 4)},
-                     "tflops": tflops, "frac_tensor": tflops / fp4_peak, "peak_tensor": fp4_peak,
-                     "peak_tensor_source": tensor_src, "frac_tensor_sustained": tflops / fp4_sustained,
-                     "frac_tensor_nominal": tflops / NOMINAL_FP4_TFLOPS, "gbs": gbs,
-                     "frac_hbm": gbs / peaks["hbm_gbs"]})
+        roof = gemm_roofline(layer.gemm_flops[dominant], layer.gemm_out_bytes(dominant), dom_ms, fp4_peak,
+                             fp4_sustained, peaks["hbm_gbs"], tensor_src, peaks["source"] + " copy bandwidth")
+        roof.update({"kernel": dominant, "traffic": dom_traffic})
     else:
         achieved = layer.quant_bytes[dominant] / (dom_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
