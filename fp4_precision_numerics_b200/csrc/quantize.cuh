@@ -272,7 +272,13 @@ template <typename InT>
 __host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(cols_tt<InT>() * kColsTF * sizeof(InT)); }
 
 template <typename InT>
-__host__ __device__ constexpr uint32_t cols_smem_bytes() { return kColsRing * cols_tile_bytes<InT>() + 64 + 128; }
+__host__ __device__ constexpr uint32_t cols_stage_bytes() { return uint32_t(kColsTF * (cols_tt<InT>() / 2)); }
+
+// the ring, its barriers and the abort flag, and two token-dim code buffers
+template <typename InT>
+__host__ __device__ constexpr uint32_t cols_smem_bytes() {
+    return kColsRing * cols_tile_bytes<InT>() + 64 + 128 + 2 * cols_stage_bytes<InT>();
+}
 
 // Dual mode (DUAL): every tile is also quantised in 1x32 blocks along the
 // features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
@@ -324,6 +330,16 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
     constexpr uint32_t kTile = cols_tile_bytes<InT>();
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + kColsRing * kTile);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kColsRing * kTile + 8 * kColsRing);
+    // Token-dim codes: a lane's 16 bytes go to its own feature row, so the
+    // warp's direct store covers 32 rows with half sectors.  Except in the
+    // dual SR kernel (issue-bound, where the extra instructions cost more than
+    // the stores save), each tile's codes are staged as [feature][kTT / 2
+    // bytes] (16-byte chunk c of row r at chunk c ^ ((r >> 1) & (kTT / 32 - 1)),
+    // two buffers) and written after the tile's barrier as whole row segments.
+    constexpr bool kStageCodes = !(DUAL && SR);
+    constexpr uint32_t kStage = cols_stage_bytes<InT>();
+    constexpr int kCh = kTT / 32;
+    uint8_t* stage_base = smem + kColsRing * kTile + 64 + 128;
     const uint32_t T = uint32_t(a.rows), F = uint32_t(a.cols);
     const uint32_t ntt = (T + kTT - 1) / kTT, ntf = (F + kTF - 1) / kTF;
     const uint32_t ntiles = uint32_t(a.groups) * ntt * ntf;
@@ -404,8 +420,14 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                 const uint2 q0 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v), n0, keys, a.sr_offset);
                 const uint2 q1 = quant16_scaled<SR>(*reinterpret_cast<const float(*)[16]>(v + 16), n0 + 16, keys,
                                                     a.sr_offset);
-                *reinterpret_cast<uint4*>(a.codes + uint64_t(orow + h) * (T >> 1) + (tb >> 1)) =
-                    make_uint4(q0.x, q0.y, q1.x, q1.y);
+                if constexpr (kStageCodes) {
+                    const int fl = 2 * pr + h;
+                    *reinterpret_cast<uint4*>(stage_base + (i & 1u) * kStage + fl * (kTT / 2) +
+                                              16 * (blk ^ ((fl >> 1) & (kCh - 1)))) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                } else {
+                    *reinterpret_cast<uint4*>(a.codes + uint64_t(orow + h) * (T >> 1) + (tb >> 1)) =
+                        make_uint4(q0.x, q0.y, q1.x, q1.y);
+                }
                 const int sb = h ? sb1 : sb0;
                 if (a.scales) a.scales[uint64_t(orow + h) * S + s] = uint8_t(sb);
                 if (a.scales_mma) a.scales_mma[g * mma_group_c + mma_off32(f + h, s, nchunk_c)] = uint8_t(sb);
@@ -545,6 +567,19 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
             }
         }
         __syncthreads();  // buffer b fully read: refill it with tile i + kColsRing
+        if (kStageCodes && !*abort_flag) {
+            // the tile's token-dim codes: whole kTT/2-byte row segments; the
+            // buffer is written again two tiles later, after the next barrier
+            const uint8_t* stg = stage_base + (i & 1u) * kStage;
+#pragma unroll
+            for (int it = 0; it < kTF * kCh / cols_threads<InT>(); ++it) {
+                const int idx = it * cols_threads<InT>() + int(threadIdx.x);
+                const int fl = idx / kCh, c = idx % kCh;
+                if (f0 + fl < F && t0 + 32 * c < T)
+                    *reinterpret_cast<uint4*>(a.codes + uint64_t(g * F + f0 + fl) * (T >> 1) + ((t0 >> 1) + 16 * c)) =
+                        *reinterpret_cast<const uint4*>(stg + fl * (kTT / 2) + 16 * (c ^ ((fl >> 1) & (kCh - 1))));
+            }
+        }
         if (threadIdx.x == 0 && i + kColsRing < mine) {
             mbar_arrive_expect_tx(&full[b], kTile);
             tma_load_3d(smem + b * kTile, &tm_in, &full[b], int32_t(nxt.tf * kTF), int32_t(nxt.tt * kTT),
