@@ -270,8 +270,8 @@ class Layer:
 # commands are in profiles/moe_layer_small_dram_counters.md).  An entry must
 # go back to None when its kernel changes.
 DRAM_BYTES_FULL = {
-    "deosc_up": 4 * (663.90e6 + 243.15e6), "deosc_down": None,   # deosc_down: not yet captured with the column-of-8 kernel
-    "dual_x": 4 * (97.43e6 + 15.15e6), "dual_h": 4 * (97.42e6 + 12.05e6),
+    "deosc_up": 4 * (663.90e6 + 242.47e6), "deosc_down": 4 * (332.08e6 + 102.85e6),
+    "dual_x": 4 * (97.39e6 + 19.04e6), "dual_h": 4 * (97.39e6 + 13.97e6),
     "dual_dy_up": 4 * (194.73e6 + 67.89e6), "dual_dy_down": 4 * (97.43e6 + 11.64e6),
     "fprop_up": 4 * (97.13e6 + 332.59e6), "fprop_down": 4 * (61.32e6 + 135.22e6),
     "dgrad_up": 4 * (122.53e6 + 149.11e6), "dgrad_down": 4 * (61.32e6 + 137.45e6),
