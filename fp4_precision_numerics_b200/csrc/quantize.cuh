@@ -274,6 +274,14 @@ __host__ __device__ constexpr uint32_t cols_tile_bytes() { return uint32_t(cols_
 template <typename InT>
 __host__ __device__ constexpr uint32_t cols_stage_bytes() { return uint32_t(kColsTF * (cols_tt<InT>() / 2)); }
 
+// Token-dim code staging: byte offset, inside one tile's buffer, of the 16
+// code bytes of the tile's feature row fl and 32-token block c.  Rows are
+// kTT/2 bytes; chunk c of row fl sits at chunk c ^ ((fl >> 1) & (kTT/32 - 1)).
+template <typename InT>
+__host__ __device__ constexpr int cols_stage_off(int fl, int c) {
+    return fl * (cols_tt<InT>() / 2) + 16 * (c ^ ((fl >> 1) & (cols_tt<InT>() / 32 - 1)));
+}
+
 // the ring, its barriers and the abort flag, and two token-dim code buffers
 template <typename InT>
 __host__ __device__ constexpr uint32_t cols_smem_bytes() {
@@ -334,8 +342,8 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
     // warp's direct store covers 32 rows with half sectors.  Except in the
     // dual SR kernel (issue-bound, where the extra instructions cost more than
     // the stores save), each tile's codes are staged as [feature][kTT / 2
-    // bytes] (16-byte chunk c of row r at chunk c ^ ((r >> 1) & (kTT / 32 - 1)),
-    // two buffers) and written after the tile's barrier as whole row segments.
+    // bytes] (cols_stage_off, two buffers) and written after the tile's
+    // barrier as whole row segments.
     constexpr bool kStageCodes = !(DUAL && SR);
     constexpr uint32_t kStage = cols_stage_bytes<InT>();
     constexpr int kCh = kTT / 32;
@@ -422,8 +430,8 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                                                     a.sr_offset);
                 if constexpr (kStageCodes) {
                     const int fl = 2 * pr + h;
-                    *reinterpret_cast<uint4*>(stage_base + (i & 1u) * kStage + fl * (kTT / 2) +
-                                              16 * (blk ^ ((fl >> 1) & (kCh - 1)))) = make_uint4(q0.x, q0.y, q1.x, q1.y);
+                    *reinterpret_cast<uint4*>(stage_base + (i & 1u) * kStage + cols_stage_off<InT>(fl, blk)) =
+                        make_uint4(q0.x, q0.y, q1.x, q1.y);
                 } else {
                     *reinterpret_cast<uint4*>(a.codes + uint64_t(orow + h) * (T >> 1) + (tb >> 1)) =
                         make_uint4(q0.x, q0.y, q1.x, q1.y);
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
                 const int fl = idx / kCh, c = idx % kCh;
                 if (f0 + fl < F && t0 + 32 * c < T)
                     *reinterpret_cast<uint4*>(a.codes + uint64_t(g * F + f0 + fl) * (T >> 1) + ((t0 >> 1) + 16 * c)) =
-                        *reinterpret_cast<const uint4*>(stg + fl * (kTT / 2) + 16 * (c ^ ((fl >> 1) & (kCh - 1))));
+                        *reinterpret_cast<const uint4*>(stg + cols_stage_off<InT>(fl, c));
             }
         }
         if (threadIdx.x == 0 && i + kColsRing < mine) {
@@ -865,6 +873,18 @@ __device__ __forceinline__ void nib_swap(uint32_t (&w)[4]) {
     }
 }
 
+// W^T staging of the column-of-blocks CTA.  Lane l of the warp of block row
+// bil (block column bjl) leaves its 16 W^T bytes in slot
+// coal_wt_slot(bjl, l, bil); thread t writes slot t out, which holds piece
+// t % kCoalBlkRows of the row pair index t / kCoalBlkRows.  The piece of lane
+// l of block column bj is W^T row coal_wt_row(bj, l) of its group.
+__host__ __device__ constexpr int coal_wt_slot(int bjl, int lane, int bil) {
+    return (bjl * 32 + lane) * kCoalBlkRows + bil;
+}
+__host__ __device__ constexpr int64_t coal_wt_row(int64_t bj, int lane) {
+    return bj * 32 + 4 * (lane & 7) + (lane >> 3);
+}
+
 // One 32x32 block of the coalesced layout (lane 8q + c holds rows 4k + q,
 // elements 4c..4c+3): block maximum, scale, codes, de-oscillation state,
 // and the block's W^T codes, which go to *ct (16 bytes of W^T row
@@ -1011,8 +1031,8 @@ __global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __g
     const int bil = warp / kCoalBlkCols, bjl = warp % kCoalBlkCols;
     const int64_t bi = int64_t(ti) * kCoalBlkRows + bil;
     const int64_t bj = int64_t(tj) * kCoalBlkCols + bjl;
-    __shared__ uint4 s_ct[kCoalBlkCols][32][kCoalBlkRows];   // W^T pieces: [block column][lane][block row]
-    if (g < a.groups && bi < nbr && bj < nbc) coal_block<InT, DEOSC>(a, g, bi, bj, lane, &s_ct[bjl][lane][bil]);
+    __shared__ uint4 s_ct[kCoalBlkCols * 32 * kCoalBlkRows];   // W^T pieces, by coal_wt_slot
+    if (g < a.groups && bi < nbr && bj < nbc) coal_block<InT, DEOSC>(a, g, bi, bj, lane, &s_ct[coal_wt_slot(bjl, lane, bil)]);
     if (!a.codes_t || g >= a.groups) return;   // uniform over the CTA
     __syncthreads();
     // thread t writes piece t % kCoalBlkRows of W^T row t / kCoalBlkRows, so
@@ -1023,8 +1043,8 @@ __global__ void __launch_bounds__(kCoalWarps * 32) quant2d_coal_kernel(const __g
     const int64_t bis = int64_t(ti) * kCoalBlkRows + p;
     const int64_t bjs = int64_t(tj) * kCoalBlkCols + wb;
     if (bis >= nbr || bjs >= nbc) return;
-    const int64_t tr = g * C + bjs * 32 + 4 * (l & 7) + (l >> 3);   // row of W^T
-    *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + bis * 16) = s_ct[wb][l][p];
+    const int64_t tr = g * C + coal_wt_row(bjs, l);   // row of W^T
+    *reinterpret_cast<uint4*>(a.codes_t + tr * (R >> 1) + bis * 16) = s_ct[threadIdx.x];   // slot (wb, l, p)
 }
 
 // ---------------------------------------------------------------------------

@@ -289,3 +289,18 @@ def test_pair_gemm_unit_walk_matches_direct_decomposition(tmp_path):
                     "-o", exe, src, "-lcuda"], check=True)
     out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
     assert out.startswith("ok") and int(out.split()[1]) > 10 ** 6, out
+
+
+def test_staging_index_maps_match_the_direct_stores(tmp_path):
+    """The shared-memory staging of the token-dim codes (quant1d_cols_kernel)
+    and of the W^T codes (quant2d_coal_kernel): every piece lands in its own
+    16-byte slot, and the cooperative store writes each slot to the row and
+    bytes of the direct store of the lane that filled it; checked by a host
+    program built from the kernels' header."""
+    src = os.path.join(ROOT, "tests", "native", "staging_check.cu")
+    exe = str(tmp_path / "staging_check")
+    subprocess.run(["nvcc", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-I",
+                    os.path.join(ROOT, "fp4_precision_numerics_b200", "csrc"), "-I", os.path.join(ROOT, "include"),
+                    "-o", exe, src, "-lcuda"], check=True)
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    assert out.startswith("ok") and int(out.split()[1]) > 3000, out
