@@ -445,8 +445,8 @@ __global__ void __launch_bounds__(256, 2) quant1d_cols_kernel(const __grid_const
             // the same tile, 1x32 blocks along the features
             constexpr int kChunks16 = 32 * int(sizeof(InT)) / 16;   // 16-byte chunks per 32-element block
             const uint8_t* tile = smem + b * kTile;
-#pragma unroll 1
-            for (int e = threadIdx.x; e < kTT * (kTF / 32); e += blockDim.x) {
+#pragma unroll   // compile-time trip count (the launch has cols_threads threads)
+            for (int e = int(threadIdx.x); e < kTT * (kTF / 32); e += cols_threads<InT>()) {
                 const int rr = e / (kTF / 32), fb = e % (kTF / 32);
                 const uint32_t t = t0 + rr, fc = f0 + 32 * fb;
                 if (!got || t >= T || fc >= F) continue;
