@@ -310,7 +310,7 @@ KERNELS = ["deosc_up", "deosc_down", "dual_x", "fprop_up", "dual_h", "fprop_down
 # Thread instructions per element of the stochastic-rounding quantisers:
 # ncu smsp__inst_executed.sum x 32 / elements of one launch (profiles/ gives
 # the commands).  An entry must go back to None when its kernel changes.
-SR_INST_PER_ELEMENT = {"dual_dy_up": 20.84, "dual_dy_down": 21.19, "rows_sr": 10.39}
+SR_INST_PER_ELEMENT = {"dual_dy_up": 20.59, "dual_dy_down": 20.94, "rows_sr": 10.39}
 SMSP_PER_SM = 4          # warp schedulers per SM, each issuing one warp instruction per cycle
 
 
