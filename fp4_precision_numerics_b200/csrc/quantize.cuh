@@ -288,10 +288,6 @@ __host__ __device__ constexpr uint32_t cols_smem_bytes() {
     return kColsRing * cols_tile_bytes<InT>() + 64 + 128 + 2 * cols_stage_bytes<InT>();
 }
 
-// Dual mode (DUAL): every tile is also quantised in 1x32 blocks along the
-// features (the layout of quant1d_rows_kernel) into a.r_*, so one read of
-// the input feeds both the contraction-dim codes and the token-dim codes.
-// Each thread takes two of the tile's (token row, 32-feature block) pairs.
 // Tile walk of a persistent CTA: tiles first, first + step, ... of a
 // [groups][token tiles][feature tiles] grid, kept as (g, tt, tf) and advanced
 // with adds and one conditional wrap per level (no division in the loop).
